@@ -1,0 +1,476 @@
+#!/usr/bin/env python
+"""Benchmark of the Engram hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+engram_hash_gather (n-gram hash + gather of 16 table rows per token),
+engram_gate_fwd, engram_gate_bwd and engram_grad_w_reduce (and, on more than
+one GPU, an NCCL all-reduce of dwh/dwe, the path's one exchange step).
+
+Default workload ("full_path"): 4 x 16384 = 65536 tokens with Zipf(1.1) ids
+over a 129280-id vocabulary, 2 n-gram layers (2-, 3-grams) x 8 tables of
+~1,000,003 rows x 64 bf16 (2.05 GB), gate at H = 7168 with x, k, v and the
+upstream gradient drawn N(0,1) in bf16.  Every input is larger than the 126 MB
+L2 (each gate tensor is 940 MB), so no L2 flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  With --impl reference the fp64 CPU oracle is
+timed instead, on a bounded sample of tokens per step.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Engram gate fwd+bwd tokens/s and HBM GB/s (% of B200 peak) at H=7168"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["engram_conditional_memory_hash_b200/csrc/gate_kernels.cuh",
+                  "engram_conditional_memory_hash_b200/csrc/hash_gather.cuh",
+                  "engram_conditional_memory_hash_b200/csrc/common.cuh",
+                  "engram_conditional_memory_hash_b200/csrc/engram_abi.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+# ------------------------------------------------------------------ helpers --
+
+def algorithmic_bytes(T: int, H: int, L: int, J: int, D: int, G: int) -> dict:
+    """Bytes each kernel must move per launch (the minimum: every input read
+    once, every output written once; table rows counted per gathered row)."""
+    rows = T * L * J
+    return {
+        # tokens read + idx written + rows read + rows written
+        "hash_gather": T * 8 + rows * 8 + 2 * rows * D * 2,
+        # x, k, v read; out written; gate written; wh, we read
+        "gate_fwd": T * (4 * 2 * H + 4) + 2 * 2 * H,
+        # g, x, k, v read; dx, dk, dv written; partial rows written; wh, we read
+        "gate_bwd": T * 7 * 2 * H + G * 4 * H + 2 * 2 * H,
+        # partial rows read; dwh, dwe written; wh, we read
+        "grad_w_reduce": G * 4 * H + 2 * 4 * H + 2 * 2 * H,
+    }
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(kernel: str, units_per_launch: int):
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    e = d.get(kernel)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    per_unit = e["dram_bytes"] / e["units"]
+    return per_unit * units_per_launch
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.idx)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0: float, t1: float):
+        rows = [s for (t, s) in self.samples if t0 <= t <= t1] or [s for (_, s) in self.samples]
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+# --------------------------------------------------------- CPU oracle timing --
+
+def oracle_sample_rate(w, hin, gin, n_tokens: int, threads: int = 0):
+    """Time the oracle (as it stands) on the first n_tokens of the workload:
+    hash + gather + gate forward + gate backward with weight gradients.
+    Returns (tokens/s, seconds, threads used)."""
+    import oracle
+    o = oracle.default()
+    if threads:
+        o.set_threads(threads)
+    S = w.S
+    nseq = max(1, n_tokens // S) if n_tokens >= S else 1
+    ntok_hash = nseq * S if n_tokens >= S else n_tokens
+    toks = hin["tokens"][:nseq] if n_tokens >= S else hin["tokens"][:1, :n_tokens]
+    t0 = time.perf_counter()
+    idx = o.engram_hash(toks, hin["multipliers"], hin["ngram_n"], hin["table_sizes"],
+                        pad_id=hin["pad_id"])
+    o.engram_gather(idx, hin["table_sizes"], hin["tables"], w.D)
+    t1 = time.perf_counter()
+    sub = {n: (a[:n_tokens] if a.ndim == 2 else a) for n, a in gin.items()}
+    t2 = time.perf_counter()
+    o.engram_gate_fwd(sub["x"], sub["k"], sub["v"], sub["wh"], sub["we"], eps=w.eps)
+    o.engram_gate_bwd(sub["g"], sub["x"], sub["k"], sub["v"], sub["wh"], sub["we"], eps=w.eps)
+    t3 = time.perf_counter()
+    per_token = (t1 - t0) / ntok_hash + (t3 - t2) / n_tokens
+    return 1.0 / per_token, (t1 - t0) + (t3 - t2), o.max_threads()
+
+
+def host_inputs(w, rank: int):
+    from engram_conditional_memory_hash_b200 import inputs
+    wr = dataclasses.replace(w, index=w.index + 1000 * rank)
+    return inputs.hash_inputs(wr), inputs.gate_inputs(wr)
+
+
+# ----------------------------------------------------------------- our arm --
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import engram_conditional_memory_hash_b200 as eng
+    from engram_conditional_memory_hash_b200 import dp, inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = inputs.WORKLOADS[args.workload]
+    T, H, L, J, D = w.T, w.H, w.L, w.J, w.D
+
+    t_gen = time.perf_counter()
+    hin, gin = host_inputs(w, rank)
+    t_gen = time.perf_counter() - t_gen
+
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    tokens = torch.from_numpy(hin["tokens"]).to(dev)
+    tables = to_dev(hin["tables"])
+    g = {n: to_dev(a) for n, a in gin.items()}
+    G = eng.engram_gate_bwd_num_partials(T, H)
+    idx = torch.empty((w.B, w.S, L, J), dtype=torch.int64, device=dev)
+    rows = torch.empty((w.B, w.S, L, J, D), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    gate = torch.empty((T,), dtype=torch.float32, device=dev)
+    dx, dk, dv = (torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    part = torch.empty((G, H), dtype=torch.float32, device=dev)
+    dw = torch.empty((2, H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    names = ["hash_gather", "gate_fwd", "gate_bwd", "grad_w_reduce"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        eng.engram_hash_gather(tokens, hin["multipliers"], hin["ngram_n"], hin["table_sizes"],
+                               tables, pad_id=hin["pad_id"], idx_out=idx, rows_out=rows)
+        mark(1)
+        eng.engram_gate_fwd(g["x"], g["k"], g["v"], g["wh"], g["we"], eps=w.eps, out=out, gate=gate)
+        mark(2)
+        eng.engram_gate_bwd(g["g"], g["x"], g["k"], g["v"], g["wh"], g["we"], eps=w.eps,
+                            dx=dx, dk=dk, dv=dv, w_partial=part)
+        mark(3)
+        eng.engram_grad_w_reduce(part, g["wh"], g["we"], dwh=dw[0], dwe=dw[1])
+        mark(4)
+        if world > 1:
+            dp.allreduce_weight_grads(dw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.2)
+    clocks.stop()
+    elapsed_ms = start.elapsed_time(end)
+    per_kernel_ms = {n: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs]))
+                     for i, n in enumerate(names)}
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    tokens_per_s = world * T / (ms_per_step / 1e3)
+
+    ab = algorithmic_bytes(T, H, L, J, D, G)
+    peak, peak_kind = measured_peak()
+    kern = {}
+    for n in names:
+        us = per_kernel_ms[n] * 1e3
+        gbs = ab[n] / (per_kernel_ms[n] / 1e3) / 1e9
+        kern[n] = {"us": round(us, 2), "algorithmic_bytes": ab[n], "GB/s": round(gbs, 1),
+                   "frac": round(gbs / peak, 4)}
+    step_bytes = sum(ab.values())
+    dominant = max(names, key=lambda n: per_kernel_ms[n])
+    roof = {
+        "kernel": dominant,
+        "bound": "hbm",
+        "achieved": round(kern[dominant]["GB/s"], 1),
+        "peak": peak,
+        "unit": "GB/s",
+        "frac": kern[dominant]["frac"],
+        "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+        else "fallback 6650 GB/s",
+        "traffic": committed_traffic(dominant, T),
+    }
+
+    # ---- end to end: host buffers in, host buffers out, copies timed -------
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = {n: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+               for n, a in gin.items() if n in ("x", "k", "v", "g")}
+        pin_tok = torch.from_numpy(hin["tokens"]).pin_memory()
+        host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                    for n, t in (("idx", idx), ("rows", rows), ("out", out), ("gate", gate),
+                                 ("dx", dx), ("dk", dk), ("dv", dv), ("dw", dw))}
+        dev_in = {"x": g["x"], "k": g["k"], "v": g["v"], "g": g["g"]}
+        h2d = sum(t.numel() * t.element_size() for t in pin.values()) + pin_tok.numel() * 8
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        dev_out = {"idx": idx, "rows": rows, "out": out, "gate": gate, "dx": dx, "dk": dk,
+                   "dv": dv, "dw": dw}
+
+        def e2e_step():
+            tokens.copy_(pin_tok, non_blocking=True)
+            for n, t in pin.items():
+                dev_in[n].copy_(t, non_blocking=True)
+            step()
+            for n, t in host_out.items():
+                t.copy_(dev_out[n], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": round(world * T / (e_ms / args.e2e_steps / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": args.e2e_steps,
+               "path": "pinned host inputs -> H2D -> C-ABI calls -> D2H of every output"}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) -------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = 64
+        rate, secs, cores = oracle_sample_rate(w, hin, gin, n)
+        target = args.cpu_seconds
+        if secs < target:
+            n = int(min(w.T, max(n, n * target / max(secs, 1e-3))))
+            rate, secs, cores = oracle_sample_rate(w, hin, gin, n)
+        cpu = {"value": round(rate, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {n} tokens of the workload (hash+gather, gate fwd+bwd with "
+                         f"weight gradients), {secs:.1f} s of fp64 CPU work"}
+
+    clk = clocks.summary(wall0, wall1)
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(tokens_per_s, 1),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded numpy PCG64: N(0,1) bf16 gate tensors, Zipf(1.1) ids, "
+                    "N(0,1) bf16 tables)",
+            "config": {
+                "workload": f"{w.name}: {w.B}x{w.S} tokens, hash+gather over {L * J} tables of "
+                            f"~1M rows x {D} bf16, gate fwd+bwd at H={H}",
+                "T": T, "H": H, "L": L, "J": J, "D": D, "G": G,
+                "l2": "inputs larger than L2 (940 MB per gate tensor, 2.05 GB tables); no flush",
+                "parallelism": f"dp{world}" if world > 1 else "single GPU",
+            },
+            "hbm_gbs": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
+            "hbm_frac": round(step_bytes / (ms_per_step / 1e3) / 1e9 / peak, 4),
+            "gate_fwd_bwd_tokens_per_s": round(
+                world * T / ((per_kernel_ms["gate_fwd"] + per_kernel_ms["gate_bwd"]
+                              + per_kernel_ms["grad_w_reduce"]) / 1e3), 1),
+            "kernels": kern,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk,
+            "input_generation_s": round(t_gen, 1),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------- reference arm --
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from engram_conditional_memory_hash_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    hin, gin = host_inputs(w, 0)
+    n = args.ref_tokens
+    rates, secs_all = [], []
+    cores = 0
+    for i in range(args.warmup + args.steps):
+        rate, secs, cores = oracle_sample_rate(w, hin, gin, n)
+        if i >= args.warmup:
+            rates.append(rate)
+            secs_all.append(secs)
+    value = float(np.median(rates))
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * float(np.median(secs_all)), 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the GPU arm)",
+        "config": {"workload": f"{w.name}: {w.B}x{w.S} tokens, gate H={w.H}", "T": w.T, "H": w.H},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"first {n} tokens of the workload per step (hash+gather, gate "
+                                   "fwd+bwd with weight gradients)"},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="full_path")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=32)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,379 @@
+// C ABI of the Engram hot path: argument checks, launch configuration and
+// launches.  Declared in include/engram.h, which documents every call.
+//
+// All kernels live in this one translation unit (included below) so that the
+// device error word has a single definition.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "engram.h"
+
+#include "common.cuh"
+#include "gate_kernels.cuh"
+#include "hash_gather.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+engram_status_t fail(engram_status_t st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+engram_status_t cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(ENGRAM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Per-device facts used to size the launches, read once per device.
+struct DeviceInfo {
+    int sms = 0;
+    int smem_optin = 0;     // largest dynamic shared memory a CTA may opt into
+    int smem_per_sm = 0;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_ready[kMaxDevices];
+
+engram_status_t device_info(DeviceInfo *out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(ENGRAM_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_dev_ready[dev]) {
+        DeviceInfo d;
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+                cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                                        dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        g_dev[dev] = d;
+        g_dev_ready[dev] = true;
+    }
+    *out = g_dev[dev];
+    return ENGRAM_OK;
+}
+
+// ------------------------------------------------------------ gate shape ----
+
+constexpr int kGateMaxH = 8192;
+constexpr int kGateMaxStages = 8;
+
+struct GateLaunch {
+    int maxv = 1;       // 16-byte column vectors per thread
+    int threads = 32;
+    int nstage = 2;
+    size_t smem = 0;
+    int ctas_per_sm = 1;
+};
+
+// Thread count and pipeline depth of a gate kernel streaming `ntensors` rows
+// of H bf16 per token.
+engram_status_t gate_plan(const DeviceInfo &d, int H, int ntensors, GateLaunch *g)
+{
+    const int nvec = H / 8;
+    g->maxv = nvec <= engram::kGateMaxThreads ? 1 : 2;
+    g->threads = ((nvec + g->maxv - 1) / g->maxv + 31) / 32 * 32;
+    const size_t stage = (size_t)ntensors * H * 2;
+    const size_t fixed = engram::kGateRedBytes;
+    int ns = (int)(((size_t)d.smem_optin - fixed) / (stage + 8));
+    ns = std::min(ns, kGateMaxStages);
+    if (ns < 2)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "H=%d: two pipeline stages need %zu B of shared memory",
+                    H, 2 * (stage + 8) + fixed);
+    g->nstage = ns;
+    g->smem = engram::gate_smem_bytes(H, ntensors, ns);
+    return ENGRAM_OK;
+}
+
+// Resident CTAs per SM of `kernel` with the plan's block and shared memory.
+template <typename K>
+engram_status_t gate_occupancy(K kernel, GateLaunch *g)
+{
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g->smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, g->threads, g->smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (n < 1) return fail(ENGRAM_ERR_UNSUPPORTED, "gate kernel does not fit on an SM");
+    g->ctas_per_sm = n;
+    return ENGRAM_OK;
+}
+
+// Forward / backward plan for H, including occupancy.
+engram_status_t gate_fwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
+{
+    engram_status_t st = gate_plan(d, H, 3, g);
+    if (st != ENGRAM_OK) return st;
+    return g->maxv == 1 ? gate_occupancy(engram::gate_fwd_kernel<1>, g)
+                        : gate_occupancy(engram::gate_fwd_kernel<2>, g);
+}
+
+engram_status_t gate_bwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
+{
+    engram_status_t st = gate_plan(d, H, 4, g);
+    if (st != ENGRAM_OK) return st;
+    return g->maxv == 1 ? gate_occupancy(engram::gate_bwd_kernel<1>, g)
+                        : gate_occupancy(engram::gate_bwd_kernel<2>, g);
+}
+
+engram_status_t check_gate_common(int64_t T, int32_t H, float eps, float scalar)
+{
+    if (T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+    if (T > (int64_t(1) << 40)) return fail(ENGRAM_ERR_UNSUPPORTED, "T=%lld too large", (long long)T);
+    if (H < 8 || H % 8 != 0 || H > kGateMaxH)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "H=%d: must be a multiple of 8 in [8, %d]", H, kGateMaxH);
+    if (!std::isfinite(eps) || eps < 0.f) return fail(ENGRAM_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    if (!std::isfinite(scalar)) return fail(ENGRAM_ERR_INVALID_ARG, "scalar must be finite");
+    return ENGRAM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int engram_abi_version(void) { return 1; }
+
+const char *engram_status_string(engram_status_t status)
+{
+    switch (status) {
+    case ENGRAM_OK: return "ok";
+    case ENGRAM_ERR_INVALID_ARG: return "invalid argument";
+    case ENGRAM_ERR_UNSUPPORTED: return "unsupported size";
+    case ENGRAM_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+const char *engram_last_error(void) { return g_last_error; }
+
+// ------------------------------------------------------------ hash/gather ----
+
+engram_status_t engram_hash_gather(const int64_t *tokens, int64_t B, int64_t S,
+                                   const uint64_t *multipliers, const int32_t *ngram_n, int32_t L,
+                                   int32_t n_max, const int64_t *table_sizes, int32_t J,
+                                   const void *tables, int32_t D, int64_t pad_id, int64_t *idx_out,
+                                   void *rows_out, engram_stream_t stream)
+{
+    using engram::HashParams;
+    if (B < 0 || S < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B=%lld, S=%lld", (long long)B, (long long)S);
+    if (!multipliers || !ngram_n || !table_sizes)
+        return fail(ENGRAM_ERR_INVALID_ARG, "multipliers, ngram_n and table_sizes are required");
+    if (L < 1 || L > engram::kHashMaxL) return fail(ENGRAM_ERR_UNSUPPORTED, "L=%d not in [1, %d]", L, engram::kHashMaxL);
+    if (J < 1 || J > engram::kHashMaxJ) return fail(ENGRAM_ERR_UNSUPPORTED, "J=%d not in [1, %d]", J, engram::kHashMaxJ);
+    if (n_max < 1 || n_max > engram::kHashMaxN)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "n_max=%d not in [1, %d]", n_max, engram::kHashMaxN);
+    if (B > 0 && S > 0 && B > (int64_t(1) << 40) / S) return fail(ENGRAM_ERR_UNSUPPORTED, "B*S too large");
+    const int64_t T = B * S;
+    if (T > 0 && !idx_out && !rows_out)
+        return fail(ENGRAM_ERR_INVALID_ARG, "idx_out and rows_out are both NULL");
+    if (rows_out && (D < 8 || D > 256 || D % 8 != 0))
+        return fail(ENGRAM_ERR_UNSUPPORTED, "D=%d: must be a multiple of 8 in [8, 256]", D);
+
+    HashParams p;
+    std::memset(&p, 0, sizeof p);
+    p.B = B;
+    p.S = S;
+    p.pad_id = pad_id;
+    p.L = L;
+    p.J = J;
+    p.D = rows_out ? D : 8;
+    int64_t total_rows = 0;
+    for (int l = 0; l < L; ++l) {
+        if (ngram_n[l] < 1 || ngram_n[l] > n_max)
+            return fail(ENGRAM_ERR_INVALID_ARG, "ngram_n[%d]=%d not in [1, n_max=%d]", l, ngram_n[l], n_max);
+        p.ngram_n[l] = ngram_n[l];
+        for (int i = 0; i < n_max; ++i) p.mult[l][i] = multipliers[(int64_t)l * n_max + i];
+        for (int j = 0; j < J; ++j) {
+            const int q = l * J + j;
+            const int64_t P = table_sizes[q];
+            if (P < 1) return fail(ENGRAM_ERR_INVALID_ARG, "table_sizes[%d]=%lld < 1", q, (long long)P);
+            p.P[q] = (uint64_t)P;
+            p.inv[q] = ~uint64_t(0) / (uint64_t)P;
+            p.row0[q] = total_rows;
+            // the gather addresses rows of the concatenated tables with 64-bit
+            // offsets of D * 2 bytes: keep the row count well inside that
+            if (rows_out && P > (int64_t(1) << 48) - total_rows)
+                return fail(ENGRAM_ERR_UNSUPPORTED, "total table rows exceed 2^48");
+            total_rows += rows_out ? P : 0;
+        }
+    }
+    if (T == 0) return ENGRAM_OK;
+    if (!tokens) return fail(ENGRAM_ERR_INVALID_ARG, "tokens is NULL");
+    if (!aligned(tokens, 8)) return fail(ENGRAM_ERR_INVALID_ARG, "tokens must be 8-byte aligned");
+    if (idx_out && !aligned(idx_out, 8)) return fail(ENGRAM_ERR_INVALID_ARG, "idx_out must be 8-byte aligned");
+    if (rows_out) {
+        if (!tables) return fail(ENGRAM_ERR_INVALID_ARG, "tables is NULL");
+        if (!aligned(tables, 16) || !aligned(rows_out, 16))
+            return fail(ENGRAM_ERR_INVALID_ARG, "tables and rows_out must be 16-byte aligned");
+    }
+
+    DeviceInfo dev;
+    engram_status_t st = device_info(&dev);
+    if (st != ENGRAM_OK) return st;
+
+    const int64_t ngroups = T * L;
+    const int64_t groups_per_block = engram::kHashThreads / 8;
+    int64_t blocks = (ngroups + groups_per_block - 1) / groups_per_block;
+    blocks = std::min<int64_t>(blocks, (int64_t)dev.sms * 64);
+    const int chunks = p.D / 8;
+    const int cpl = (chunks + 7) / 8;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const uint4 *tab = static_cast<const uint4 *>(tables);
+    uint4 *rows = static_cast<uint4 *>(rows_out);
+    if (cpl <= 1)
+        engram::hash_gather_kernel<1><<<(unsigned)blocks, engram::kHashThreads, 0, s>>>(tokens, tab, idx_out, rows, p);
+    else if (cpl <= 2)
+        engram::hash_gather_kernel<2><<<(unsigned)blocks, engram::kHashThreads, 0, s>>>(tokens, tab, idx_out, rows, p);
+    else
+        engram::hash_gather_kernel<4><<<(unsigned)blocks, engram::kHashThreads, 0, s>>>(tokens, tab, idx_out, rows, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "hash_gather launch");
+    return ENGRAM_OK;
+}
+
+// ---------------------------------------------------------------- gate fwd ----
+
+engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, const void *wh,
+                                const void *we, int64_t T, int32_t H, float eps, float scalar,
+                                void *out, float *gate, engram_stream_t stream)
+{
+    engram_status_t st = check_gate_common(T, H, eps, scalar);
+    if (st != ENGRAM_OK) return st;
+    if (T == 0) return ENGRAM_OK;
+    if (!x || !k || !v || !wh || !we || !out)
+        return fail(ENGRAM_ERR_INVALID_ARG, "x, k, v, wh, we and out are required");
+    if (!aligned(x, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(wh, 16) || !aligned(we, 16) ||
+        !aligned(out, 16))
+        return fail(ENGRAM_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+    if (gate && !aligned(gate, 4)) return fail(ENGRAM_ERR_INVALID_ARG, "gate must be 4-byte aligned");
+
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != ENGRAM_OK) return st;
+    GateLaunch g;
+    if ((st = gate_fwd_plan(dev, H, &g)) != ENGRAM_OK) return st;
+    const int64_t grid = std::min<int64_t>(T, (int64_t)dev.sms * g.ctas_per_sm);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    auto args = [&](auto kern) -> engram_status_t {
+        kern<<<(unsigned)grid, g.threads, g.smem, s>>>(
+            static_cast<const uint4 *>(x), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+            static_cast<const uint4 *>(wh), static_cast<const uint4 *>(we), T, H, eps, scalar,
+            static_cast<uint4 *>(out), gate, g.nstage);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "gate_fwd launch");
+        return ENGRAM_OK;
+    };
+    return g.maxv == 1 ? args(engram::gate_fwd_kernel<1>) : args(engram::gate_fwd_kernel<2>);
+}
+
+// ---------------------------------------------------------------- gate bwd ----
+
+int64_t engram_gate_bwd_num_partials(int64_t T, int32_t H)
+{
+    if (H < 8 || H % 8 != 0 || H > kGateMaxH) {
+        fail(ENGRAM_ERR_UNSUPPORTED, "H=%d: must be a multiple of 8 in [8, %d]", H, kGateMaxH);
+        return -1;
+    }
+    DeviceInfo dev;
+    if (device_info(&dev) != ENGRAM_OK) return -1;
+    GateLaunch g;
+    if (gate_bwd_plan(dev, H, &g) != ENGRAM_OK) return -1;
+    const int64_t full = (int64_t)dev.sms * g.ctas_per_sm;
+    return std::max<int64_t>(1, std::min<int64_t>(T, full));
+}
+
+engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void *k, const void *v,
+                                const void *wh, const void *we, int64_t T, int32_t H, float eps,
+                                float scalar, void *dx, void *dk, void *dv, float *w_partial, int64_t G,
+                                engram_stream_t stream)
+{
+    engram_status_t st = check_gate_common(T, H, eps, scalar);
+    if (st != ENGRAM_OK) return st;
+    if (!wh || !we || !w_partial)
+        return fail(ENGRAM_ERR_INVALID_ARG, "wh, we and w_partial are required");
+    // with T == 0 the kernel only writes zero partial rows; the token tensors
+    // may then be empty (NULL)
+    if (T > 0 && (!grad_out || !x || !k || !v || !dx || !dk || !dv))
+        return fail(ENGRAM_ERR_INVALID_ARG, "every tensor argument of engram_gate_bwd is required");
+    if (G < 1 || G > 0x7fffffff) return fail(ENGRAM_ERR_INVALID_ARG, "G=%lld not in [1, 2^31-1]", (long long)G);
+    if (!aligned(grad_out, 16) || !aligned(x, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(wh, 16) || !aligned(we, 16) || !aligned(dx, 16) || !aligned(dk, 16) ||
+        !aligned(dv, 16) || !aligned(w_partial, 16))
+        return fail(ENGRAM_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != ENGRAM_OK) return st;
+    GateLaunch g;
+    if ((st = gate_bwd_plan(dev, H, &g)) != ENGRAM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    auto args = [&](auto kern) -> engram_status_t {
+        kern<<<(unsigned)G, g.threads, g.smem, s>>>(
+            static_cast<const uint4 *>(grad_out), static_cast<const uint4 *>(x),
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<const uint4 *>(wh),
+            static_cast<const uint4 *>(we), T, H, eps, scalar, static_cast<uint4 *>(dx),
+            static_cast<uint4 *>(dk), static_cast<uint4 *>(dv), w_partial, g.nstage);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "gate_bwd launch");
+        return ENGRAM_OK;
+    };
+    return g.maxv == 1 ? args(engram::gate_bwd_kernel<1>) : args(engram::gate_bwd_kernel<2>);
+}
+
+// ----------------------------------------------------------- grad_w_reduce ----
+
+engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t G, int32_t H, const void *wh,
+                                     const void *we, float *dwh, float *dwe, engram_stream_t stream)
+{
+    if (G < 1 || G > 0x7fffffff) return fail(ENGRAM_ERR_INVALID_ARG, "G=%lld not in [1, 2^31-1]", (long long)G);
+    if (H < 1) return fail(ENGRAM_ERR_INVALID_ARG, "H=%d < 1", H);
+    if (!w_partial || !wh || !we || !dwh || !dwe)
+        return fail(ENGRAM_ERR_INVALID_ARG, "every pointer argument of engram_grad_w_reduce is required");
+    if (!aligned(w_partial, 4) || !aligned(dwh, 4) || !aligned(dwe, 4) || !aligned(wh, 2) || !aligned(we, 2))
+        return fail(ENGRAM_ERR_INVALID_ARG, "misaligned pointer");
+    const unsigned blocks = (unsigned)((H + 31) / 32);
+    engram::grad_w_reduce_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        w_partial, G, H, static_cast<const __nv_bfloat16 *>(wh), static_cast<const __nv_bfloat16 *>(we),
+        dwh, dwe);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "grad_w_reduce launch");
+    return ENGRAM_OK;
+}
+
+// ------------------------------------------------------------ diagnostics ----
+
+engram_status_t engram_read_device_error(uint32_t *code_out, int32_t clear)
+{
+    if (!code_out) return fail(ENGRAM_ERR_INVALID_ARG, "code_out is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    unsigned int v = 0;
+    e = cudaMemcpyFromSymbol(&v, engram::g_device_error, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+    if (clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(engram::g_device_error, &zero, sizeof zero);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+    }
+    *code_out = v;
+    return ENGRAM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,199 @@
+/*
+ * engram.h - C ABI of the Engram conditional-memory hot path for NVIDIA B200
+ * (sm_100a): the n-gram hash with its table-row gather, and the fused Engram
+ * gate, forward and backward, with the weight-gradient reduction.
+ *
+ * The operations are the Engram kernels listed on the page "DeepSeek 开源
+ * TileKernels：用 Python 写出逼近硬件极限的 GPU 内核" (zhichai.net/topic/177618722),
+ * section "5. Engram — 条件记忆门控": engram_hash, engram_gate_fwd/bwd,
+ * engram_fused_weight and engram_grad_w_reduce, with the gate formula
+ *
+ *     gate   = sigmoid(signed_sqrt(dot(RMSNorm(x, wh), RMSNorm(k, we)) * scalar))
+ *     output = hidden_states + gate * v
+ *     signed_sqrt(s) = sign(s) * sqrt(|s|),  scalar = 1 / sqrt(hidden_size).
+ *
+ * Conventions shared by every call:
+ *   - Device pointers point to CUDA device memory of the current device.  The
+ *     caller allocates every buffer and keeps ownership; the library allocates
+ *     nothing and keeps no state between calls.
+ *   - Every compute call is asynchronous on `stream` (NULL: the legacy default
+ *     stream) and never synchronises.  Outputs are valid once the stream has
+ *     reached the call.
+ *   - "bf16" tensors are contiguous, row-major arrays of IEEE bfloat16.  Every
+ *     bf16 tensor must start on a 16-byte boundary; H must be a multiple of 8
+ *     (one 16-byte vector holds 8 bf16 values).
+ *   - Errors: arguments are checked before anything is launched; a failing
+ *     check returns ENGRAM_ERR_INVALID_ARG (bad pointer, size or alignment) or
+ *     ENGRAM_ERR_UNSUPPORTED (a size this build does not handle) and launches
+ *     nothing.  A failing CUDA runtime call returns ENGRAM_ERR_CUDA.  The
+ *     message of the last failure on the calling thread is returned by
+ *     engram_last_error().  Kernels never trap; a pipeline wait that exceeds
+ *     its time limit records a code that engram_read_device_error() reports.
+ */
+#ifndef ENGRAM_H
+#define ENGRAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ENGRAM_API __attribute__((visibility("default")))
+#else
+#define ENGRAM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+struct CUstream_st;
+typedef struct CUstream_st *engram_stream_t;
+
+typedef enum {
+    ENGRAM_OK = 0,
+    ENGRAM_ERR_INVALID_ARG = 1,
+    ENGRAM_ERR_UNSUPPORTED = 2,
+    ENGRAM_ERR_CUDA = 3
+} engram_status_t;
+
+/* Codes a kernel may record in the device error word. */
+#define ENGRAM_DEVICE_ERR_PIPELINE_TIMEOUT 1u
+
+/* Version of this ABI (incremented on any incompatible change). */
+ENGRAM_API int engram_abi_version(void);
+
+/* Static description of a status code.  Never NULL. */
+ENGRAM_API const char *engram_status_string(engram_status_t status);
+
+/* Message of the last failing call made by this thread ("" if none). */
+ENGRAM_API const char *engram_last_error(void);
+
+/*
+ * engram_hash_gather - n-gram hash to embedding-table indices, then gather of
+ * the indexed table rows ("engram_hash" on the page above; the hash combines
+ * XOR and multiplication over the token sequence and maps it to indices of 8
+ * embedding tables per n-gram layer, 2 layers, up to 3-grams).
+ *
+ * For token t = (b, s), layer l and table j:
+ *     h      = XOR_{i=0}^{ngram_n[l]-1}  u64(tok(b, s-i)) * multipliers[l*n_max + i]
+ *              (products wrap modulo 2^64; tok(b, s-i) = pad_id when s-i < 0,
+ *              so the history never crosses into another sequence)
+ *     idx    = h mod table_sizes[l*J + j]          (unsigned 64-bit remainder)
+ *     row    = rows [idx] of table (l, j)
+ *
+ * tokens      device, int64 [B*S], row-major [B][S], 8-byte aligned.
+ * B, S        >= 0 (B*S == 0 launches nothing).
+ * multipliers HOST, uint64 [L*n_max]; copied into the launch, may be freed on
+ *             return.  Entries beyond ngram_n[l] in a row are ignored.
+ * ngram_n     HOST, int32 [L], each in [1, n_max].
+ * L           number of n-gram layers, 1..4.     n_max  1..8.
+ * table_sizes HOST, int64 [L*J], rows of table (l, j) at l*J+j, each >= 1.
+ * J           tables per layer, 1..16.
+ * tables      device, bf16, the L*J tables stored one after another in
+ *             (l, j) order, each table_sizes[l*J+j] rows of D values;
+ *             16-byte aligned.  Needed only when rows_out != NULL.
+ * D           row width in bf16 values: a multiple of 8, 8..256.
+ * pad_id      token id used for positions before the start of a sequence.
+ * idx_out     device, int64 [B*S*L*J] laid out [t][l][j], 8-byte aligned,
+ *             or NULL to skip writing indices.
+ * rows_out    device, bf16 [B*S*L*J*D] laid out [t][l][j][D], 16-byte
+ *             aligned, or NULL to skip the gather (idx_out and rows_out may
+ *             not both be NULL when B*S > 0).  With rows_out the tables may
+ *             hold at most 2^48 rows in total; without it table sizes may be
+ *             any positive int64.
+ */
+ENGRAM_API engram_status_t engram_hash_gather(const int64_t *tokens, int64_t B, int64_t S,
+                                   const uint64_t *multipliers, const int32_t *ngram_n,
+                                   int32_t L, int32_t n_max, const int64_t *table_sizes,
+                                   int32_t J, const void *tables, int32_t D, int64_t pad_id,
+                                   int64_t *idx_out, void *rows_out, engram_stream_t stream);
+
+/*
+ * engram_gate_fwd - fused Engram gate forward ("engram_gate_fwd" on the page
+ * above: RMSNorm, signed-sqrt activation and sigmoid gate fused), with the
+ * fused weight w = wh * we ("engram_fused_weight") formed inside the kernel:
+ *     rx   = (mean_j x_j^2 + eps)^(-1/2),  rk = (mean_j k_j^2 + eps)^(-1/2)
+ *     s    = rx * rk * sum_j x_j k_j wh_j we_j * scalar
+ *     gate = sigmoid(sign(s) sqrt(|s|)),   out = x + gate * v
+ * Accumulation is fp32; out is rounded to bf16 (nearest even).
+ *
+ * x, k, v     device, bf16 [T*H], row-major [T][H], 16-byte aligned.
+ * wh, we      device, bf16 [H], 16-byte aligned.
+ * T           >= 0 tokens (0 launches nothing; the pointers may then be NULL).
+ * H           hidden size: multiple of 8, 8..8192.
+ * eps         >= 0, finite.   scalar  finite (normally 1/sqrt(H)).
+ * out         device, bf16 [T*H], 16-byte aligned (may not alias the inputs).
+ * gate        device, fp32 [T], 4-byte aligned, or NULL to skip it.
+ */
+ENGRAM_API engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, const void *wh,
+                                const void *we, int64_t T, int32_t H, float eps, float scalar,
+                                void *out, float *gate, engram_stream_t stream);
+
+/*
+ * engram_gate_bwd_num_partials - the recommended row count G of the
+ * weight-gradient partial buffer of engram_gate_bwd on the current device
+ * (one persistent CTA per partial row).  Returns a value >= 1, or -1 with
+ * engram_last_error() set when no CUDA device can be queried.
+ */
+ENGRAM_API int64_t engram_gate_bwd_num_partials(int64_t T, int32_t H);
+
+/*
+ * engram_gate_bwd - backward of engram_gate_fwd with respect to x, k, v and,
+ * in partial form, wh and we ("engram_gate_bwd").  The per-token statistics
+ * are recomputed from x and k; nothing is saved from the forward.  With
+ * g = grad_out, d = rx*rk*sum_j x_j k_j w_j, w = wh*we and
+ *     du = (sum_j g_j v_j) * gate * (1 - gate)
+ *     dd = du / (2 sqrt(max(|s|, 1e-6))) * scalar,    c = dd * rx * rk
+ *     dx_j = g_j + c w_j k_j - dd d rx^2 x_j / H
+ *     dk_j = c w_j x_j - dd d rk^2 k_j / H
+ *     dv_j = gate * g_j
+ *     w_partial[p][j] = sum over the tokens t of partial row p of c_t x_tj k_tj
+ * CTA p of G handles tokens p, p+G, p+2G, ... in that order, so the partials
+ * (and everything else) are bitwise reproducible for a given G.
+ *
+ * grad_out, x, k, v  device, bf16 [T*H], 16-byte aligned.
+ * wh, we             device, bf16 [H], 16-byte aligned.
+ * T >= 0, H as in engram_gate_fwd, eps/scalar as passed to the forward.
+ * dx, dk, dv         device, bf16 [T*H], 16-byte aligned (no aliasing).
+ * w_partial          device, fp32 [G*H], 16-byte aligned; fully overwritten
+ *                    (rows of CTAs without tokens are written as zeros, so
+ *                    T == 0 yields all-zero partials; the token tensors may
+ *                    then be NULL).
+ * G                  >= 1, at most 2^31 - 1 (engram_gate_bwd_num_partials()
+ *                    gives the value that fills the GPU once).
+ */
+ENGRAM_API engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void *k,
+                                const void *v, const void *wh, const void *we, int64_t T,
+                                int32_t H, float eps, float scalar, void *dx, void *dk,
+                                void *dv, float *w_partial, int64_t G, engram_stream_t stream);
+
+/*
+ * engram_grad_w_reduce - weight-gradient reduction ("engram_grad_w_reduce"):
+ *     P_j   = sum_{p=0}^{G-1} w_partial[p][j]   (fixed order, deterministic)
+ *     dwh_j = we_j * P_j,   dwe_j = wh_j * P_j
+ * which are the gradients of sum over tokens of the forward's loss with
+ * respect to wh and we.
+ *
+ * w_partial   device, fp32 [G*H] as written by engram_gate_bwd, 4-byte aligned.
+ * G >= 1, H >= 1.
+ * wh, we      device, bf16 [H], 2-byte aligned.
+ * dwh, dwe    device, fp32 [H], 4-byte aligned; overwritten, not accumulated.
+ */
+ENGRAM_API engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t G, int32_t H,
+                                     const void *wh, const void *we, float *dwh, float *dwe,
+                                     engram_stream_t stream);
+
+/*
+ * engram_read_device_error - synchronises the current device, then reads (and
+ * when `clear` is non-zero, resets) the device error word in which kernels
+ * record a pipeline wait that ran past its time limit.  *code_out receives 0
+ * or a bitwise OR of ENGRAM_DEVICE_ERR_* codes.  Diagnostic; not for hot paths.
+ */
+ENGRAM_API engram_status_t engram_read_device_error(uint32_t *code_out, int32_t clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENGRAM_H */

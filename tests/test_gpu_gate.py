@@ -1,0 +1,172 @@
+"""GPU parity of the fused Engram gate (forward, backward, weight-gradient
+reduction) against the fp64 oracle, with the tolerances stated in parity.py.
+The gate is the formula of the page "DeepSeek 开源 TileKernels"
+(zhichai.net/topic/177618722), section "5. Engram — 条件记忆门控"."""
+import numpy as np
+import pytest
+import torch
+
+import engram_conditional_memory_hash_b200 as eng
+from engram_conditional_memory_hash_b200 import inputs
+from parity import (assert_bf16_close, assert_dw_close, assert_gate_close, ill_conditioned,
+                    to_dev_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(gi):
+    return {n: to_dev_bf16(a) for n, a in gi.items()}
+
+
+def _gpu_path(t, eps=1e-6, G=None):
+    out, gate = eng.engram_gate_fwd(t["x"], t["k"], t["v"], t["wh"], t["we"], eps=eps)
+    dx, dk, dv, part = eng.engram_gate_bwd(t["g"], t["x"], t["k"], t["v"], t["wh"], t["we"],
+                                           eps=eps, G=G)
+    dwh, dwe = eng.engram_grad_w_reduce(part, t["wh"], t["we"])
+    torch.cuda.synchronize()
+    return dict(out=out, gate=gate, dx=dx, dk=dk, dv=dv, part=part, dwh=dwh, dwe=dwe)
+
+
+def _check_all(o, gi, res, eps=1e-6, rows=None):
+    """Compare every output with the oracle; rows: token sample for the
+    per-token outputs (None: all tokens)."""
+    sel = slice(None) if rows is None else rows
+    sub = {n: (a[sel] if a.ndim == 2 else a) for n, a in gi.items()}
+    ref_out, ref_gate = o.engram_gate_fwd(sub["x"], sub["k"], sub["v"], sub["wh"], sub["we"], eps=eps)
+    ref = o.engram_gate_bwd(sub["g"], sub["x"], sub["k"], sub["v"], sub["wh"], sub["we"], eps=eps,
+                            weights=rows is None)
+    ill = ill_conditioned(ref["s"])
+    pick = (lambda t: t) if rows is None else (lambda t: t[torch.from_numpy(np.asarray(rows)).cuda()])
+    rep = {
+        "out": assert_bf16_close("out", pick(res["out"]), ref_out),
+        "gate": assert_gate_close(pick(res["gate"]), ref_gate),
+        "dx": assert_bf16_close("dx", pick(res["dx"]), ref["dx"], rows_relaxed=ill),
+        "dk": assert_bf16_close("dk", pick(res["dk"]), ref["dk"], rows_relaxed=ill),
+        "dv": assert_bf16_close("dv", pick(res["dv"]), ref["dv"]),
+    }
+    if rows is None:
+        rep["dwh"] = assert_dw_close("dwh", res["dwh"], ref["dwh"])
+        rep["dwe"] = assert_dw_close("dwe", res["dwe"], ref["dwe"])
+    return rep
+
+
+def test_tiny(oracle_lib):
+    w = inputs.WORKLOADS["tiny"]
+    gi = inputs.gate_inputs(w)
+    res = _gpu_path(_dev(gi))
+    _check_all(oracle_lib, gi, res)
+    assert eng.engram_read_device_error() == 0
+
+
+@pytest.mark.parametrize("T,H", [(1, 8), (3, 264), (149, 1000 * 8 // 8 + 8), (300, 4096),
+                                 (150, 7168), (37, 8192), (5, 512), (2, 4104)])
+def test_shapes_and_ragged(oracle_lib, T, H):
+    w = inputs.Workload("ragged", 90 + H % 17, B=1, S=T, H=H, backward=True)
+    gi = inputs.gate_inputs(w)
+    res = _gpu_path(_dev(gi))
+    _check_all(oracle_lib, gi, res)
+
+
+@pytest.mark.parametrize("G", [1, 7, 148, 400])
+def test_partial_count(oracle_lib, G):
+    w = inputs.Workload("partials", 60, B=1, S=300, H=1024, backward=True)
+    gi = inputs.gate_inputs(w)
+    res = _gpu_path(_dev(gi), G=G)
+    assert tuple(res["part"].shape) == (G, 1024)
+    _check_all(oracle_lib, gi, res)
+    if G > 300:   # CTAs without tokens write zero partial rows
+        assert torch.count_nonzero(res["part"][300:]).item() == 0
+
+
+def test_closed_forms_on_gpu():
+    # x and k with disjoint supports: gate = 0.5 exactly and out = x + v/2
+    H, T = 256, 64
+    r = np.random.default_rng(3)
+    x = r.standard_normal((T, H)).astype(np.float32)
+    k = r.standard_normal((T, H)).astype(np.float32)
+    x[:, 1::2] = 0
+    k[:, 0::2] = 0
+    v = r.standard_normal((T, H)).astype(np.float32)
+    t = {n: to_dev_bf16(inputs.f32_to_bf16_bits(a)) for n, a in (("x", x), ("k", k), ("v", v))}
+    ones = torch.ones(H, dtype=torch.bfloat16, device="cuda")
+    out, gate = eng.engram_gate_fwd(t["x"], t["k"], t["v"], ones, ones)
+    torch.cuda.synchronize()
+    assert torch.all(gate == 0.5)
+    ref = (t["x"].float() + 0.5 * t["v"].float()).to(torch.bfloat16)
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    # v = 0: out = x bit for bit
+    out0, _ = eng.engram_gate_fwd(t["x"], t["k"], torch.zeros_like(t["v"]), ones, ones)
+    torch.cuda.synchronize()
+    assert torch.equal(out0.view(torch.int16), t["x"].view(torch.int16))
+    # k = x, wh = we = 1, eps = 0: gate = sigmoid(H^(1/4))
+    xx = to_dev_bf16(inputs.normal_bf16(5, 0, (T, H)))
+    _, g1 = eng.engram_gate_fwd(xx, xx, xx, ones, ones, eps=0.0)
+    torch.cuda.synchronize()
+    assert torch.allclose(g1.double(), torch.full_like(g1.double(), 0.98201379004), atol=2e-6)
+
+
+def test_deterministic(oracle_lib):
+    w = inputs.Workload("det", 70, B=1, S=500, H=7168, backward=True)
+    t = _dev(inputs.gate_inputs(w))
+    a = _gpu_path(t)
+    b = _gpu_path(t)
+    for n in ("out", "gate", "dx", "dk", "dv", "part", "dwh", "dwe"):
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+
+
+def test_misaligned_and_bad_shapes_rejected():
+    H = 64
+    x = torch.zeros(5 * H + 8, dtype=torch.bfloat16, device="cuda")
+    xs = x[4:4 + 4 * H].view(4, H)   # 8-byte offset
+    w1 = torch.ones(H, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(eng.EngramError):
+        eng.engram_gate_fwd(xs, xs, xs, w1, w1)
+    bad = torch.zeros(4, 12, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(eng.EngramError):
+        eng.engram_gate_fwd(bad, bad, bad, torch.ones(12, dtype=torch.bfloat16, device="cuda"),
+                            torch.ones(12, dtype=torch.bfloat16, device="cuda"))
+
+
+def test_empty_tokens():
+    H = 4096
+    e = torch.empty(0, H, dtype=torch.bfloat16, device="cuda")
+    w1 = torch.ones(H, dtype=torch.bfloat16, device="cuda")
+    out, gate = eng.engram_gate_fwd(e, e, e, w1, w1)
+    dx, dk, dv, part = eng.engram_gate_bwd(e, e, e, e, w1, w1, G=4)
+    dwh, dwe = eng.engram_grad_w_reduce(part, w1, w1)
+    torch.cuda.synchronize()
+    assert out.numel() == 0 and gate.numel() == 0
+    assert torch.count_nonzero(part).item() == 0 and torch.count_nonzero(dwh).item() == 0
+
+
+def test_gate_fwd_full_size(oracle_lib):
+    """Gate forward at T = 16384, H = 4096: every output against the oracle."""
+    w = inputs.WORKLOADS["gate_fwd"]
+    gi = inputs.gate_inputs(w)
+    del gi["g"]
+    t = _dev(gi)
+    out, gate = eng.engram_gate_fwd(t["x"], t["k"], t["v"], t["wh"], t["we"], eps=w.eps)
+    torch.cuda.synchronize()
+    ref_out, ref_gate = oracle_lib.engram_gate_fwd(gi["x"], gi["k"], gi["v"], gi["wh"], gi["we"],
+                                                   eps=w.eps)
+    assert_bf16_close("out", out, ref_out)
+    assert_gate_close(gate, ref_gate)
+
+
+def test_gate_fwdbwd_full_size(oracle_lib):
+    """Gate forward + backward at T = 32768, H = 7168 in the benchmark's launch
+    configuration: per-token outputs on a sample of tokens (including the most
+    ill-conditioned ones), weight gradients over all tokens."""
+    w = inputs.WORKLOADS["gate_fwdbwd"]
+    gi = inputs.gate_inputs(w)
+    res = _gpu_path(_dev(gi), eps=w.eps)
+    ref_w = oracle_lib.engram_gate_bwd(gi["g"], gi["x"], gi["k"], gi["v"], gi["wh"], gi["we"],
+                                       eps=w.eps, per_token=False)
+    assert_dw_close("dwh", res["dwh"], ref_w["dwh"])
+    assert_dw_close("dwe", res["dwe"], ref_w["dwe"])
+    r = np.random.default_rng(1)
+    worst = np.argsort(np.abs(ref_w["s"]))[:16]
+    rows = np.unique(np.concatenate([r.choice(w.T, size=496, replace=False), worst,
+                                     [0, w.T - 1]]))
+    _check_all(oracle_lib, gi, res, eps=w.eps, rows=rows)
+    assert eng.engram_read_device_error() == 0
