@@ -191,6 +191,19 @@ def oracle_sample_rate(w, hin, gin, n_tokens: int, threads: int = 0):
     return 1.0 / per_token, (t1 - t0) + (t3 - t2), o.max_threads()
 
 
+def workload(args):
+    """The named workload, optionally cut to its first --tokens tokens (whole
+    sequences where possible; used for small profiling runs)."""
+    from engram_conditional_memory_hash_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    if args.tokens and args.tokens < w.T:
+        if args.tokens >= w.S:
+            w = dataclasses.replace(w, B=args.tokens // w.S)
+        else:
+            w = dataclasses.replace(w, B=1, S=args.tokens)
+    return w
+
+
 def host_inputs(w, rank: int):
     from engram_conditional_memory_hash_b200 import inputs
     wr = dataclasses.replace(w, index=w.index + 1000 * rank)
@@ -212,7 +225,7 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    w = inputs.WORKLOADS[args.workload]
+    w = workload(args)
     T, H, L, J, D = w.T, w.H, w.L, w.J, w.D
 
     t_gen = time.perf_counter()
@@ -416,8 +429,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    from engram_conditional_memory_hash_b200 import inputs
-    w = inputs.WORKLOADS[args.workload]
+    w = workload(args)
     hin, gin = host_inputs(w, 0)
     n = args.ref_tokens
     rates, secs_all = [], []
@@ -456,10 +468,12 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="full_path")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="cut the workload to its first N tokens (profiling runs)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
