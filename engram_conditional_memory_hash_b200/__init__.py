@@ -27,14 +27,15 @@ __all__ = [
     "EngramError", "library_path", "lib", "engram_abi_version",
     "engram_hash_gather", "engram_gate_fwd", "engram_gate_bwd_num_partials",
     "engram_gate_bwd", "engram_grad_w_reduce", "engram_read_device_error",
-    "default_scalar",
+    "engram_gate_bwd_noalloc", "default_scalar",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIBRARY_NAME = "libengram_b200.so"
 EXPORTED = ("engram_abi_version", "engram_status_string", "engram_last_error",
             "engram_hash_gather", "engram_gate_fwd", "engram_gate_bwd_num_partials",
-            "engram_gate_bwd", "engram_grad_w_reduce", "engram_read_device_error")
+            "engram_gate_bwd", "engram_grad_w_reduce", "engram_read_device_error",
+            "engram_gate_bwd_noalloc")
 
 
 class EngramError(RuntimeError):
@@ -88,6 +89,9 @@ def lib() -> ctypes.CDLL:
                                           _vp, _vp, _vp, _vp, _i64, _vp]
             L.engram_grad_w_reduce.restype = ctypes.c_int
             L.engram_grad_w_reduce.argtypes = [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp]
+            L.engram_gate_bwd_noalloc.restype = ctypes.c_int
+            L.engram_gate_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _f32,
+                                                  _f32, _vp, _vp, _vp, _vp, _vp, _vp]
             L.engram_read_device_error.restype = ctypes.c_int
             L.engram_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), _i32]
             _lib = L
@@ -278,6 +282,33 @@ def engram_grad_w_reduce(w_partial, wh, we, *, dwh=None, dwe=None, stream=None):
                                     _dev(dwe, "dwe", torch.float32), _stream_ptr(stream))
     _check("engram_grad_w_reduce", st)
     return dwh, dwe
+
+
+def engram_gate_bwd_noalloc(grad_out, x, k, v, wh, we, eps: float = 1e-6,
+                            scalar: float | None = None, *, dx=None, dk=None, dv=None, dwh=None,
+                            dwe=None, stream=None):
+    """engram_gate_bwd + engram_grad_w_reduce with the library's static scratch
+    instead of a partial-row buffer, for callers that cannot allocate device
+    memory (pass every output in to allocate nothing here either).
+    Returns (dx, dk, dv bf16 [T, H], dwh, dwe fp32 [H])."""
+    T, H = _gate_shapes(x, k, v, wh, we)
+    if tuple(grad_out.shape) != (T, H):
+        raise ValueError("grad_out must be [T, H]")
+    ptrs = [_dev(t, n, torch.bfloat16) for t, n in ((grad_out, "grad_out"), (x, "x"), (k, "k"),
+                                                    (v, "v"), (wh, "wh"), (we, "we"))]
+    dx = torch.empty_like(x) if dx is None else dx
+    dk = torch.empty_like(x) if dk is None else dk
+    dv = torch.empty_like(x) if dv is None else dv
+    dwh = torch.empty((H,), dtype=torch.float32, device=x.device) if dwh is None else dwh
+    dwe = torch.empty((H,), dtype=torch.float32, device=x.device) if dwe is None else dwe
+    outs = [_dev(t, n, torch.bfloat16) for t, n in ((dx, "dx"), (dk, "dk"), (dv, "dv"))]
+    if scalar is None:
+        scalar = default_scalar(H)
+    st = lib().engram_gate_bwd_noalloc(*ptrs, T, H, float(eps), float(scalar), *outs,
+                                       _dev(dwh, "dwh", torch.float32),
+                                       _dev(dwe, "dwe", torch.float32), _stream_ptr(stream))
+    _check("engram_gate_bwd_noalloc", st)
+    return dx, dk, dv, dwh, dwe
 
 
 def engram_read_device_error(clear: bool = True) -> int:

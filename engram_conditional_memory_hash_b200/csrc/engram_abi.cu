@@ -377,3 +377,72 @@ engram_status_t engram_read_device_error(uint32_t *code_out, int32_t clear)
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------ allocation-free bwd ----
+//
+// engram_gate_bwd_noalloc: engram_gate_bwd followed by engram_grad_w_reduce
+// for callers that cannot allocate device memory (for example code running
+// under a memory-pool or graph-capture policy that forbids cudaMalloc, or a
+// host runtime whose only device buffers are the ones it was handed).  The
+// weight-gradient partial rows, the only scratch of the backward, live in the
+// fixed array below instead of a caller-provided buffer.
+
+// Scratch: partial rows of the weight-gradient reduction, at most
+// kNoAllocPartialFloats fp32 values (8 MiB).  Every GPU that loads this
+// library holds the array until the process exits.
+static constexpr size_t kNoAllocPartialFloats = size_t(1) << 21;
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocPartialFloats];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+float *g_noalloc_ptr[kMaxDevices];
+
+// Device address of g_noalloc_partials on the current device.  The name of
+// the array in host code is only a host-side stand-in, so the address is
+// looked up once per device (with that device current) and cached.
+engram_status_t noalloc_scratch(float **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(ENGRAM_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        g_noalloc_ptr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return ENGRAM_OK;
+}
+
+}  // namespace
+
+extern "C" engram_status_t engram_gate_bwd_noalloc(const void *grad_out, const void *x, const void *k,
+                                                   const void *v, const void *wh, const void *we,
+                                                   int64_t T, int32_t H, float eps, float scalar,
+                                                   void *dx, void *dk, void *dv, float *dwh,
+                                                   float *dwe, engram_stream_t stream)
+{
+    engram_status_t st = check_gate_common(T, H, eps, scalar);
+    if (st != ENGRAM_OK) return st;
+    if (!dwh || !dwe) return fail(ENGRAM_ERR_INVALID_ARG, "dwh and dwe are required");
+    if (!aligned(dwh, 4) || !aligned(dwe, 4))
+        return fail(ENGRAM_ERR_INVALID_ARG, "dwh and dwe must be 4-byte aligned");
+    const int64_t G = engram_gate_bwd_num_partials(T, H);
+    if (G < 1) return ENGRAM_ERR_CUDA;  // message set by engram_gate_bwd_num_partials
+    if ((size_t)G * (size_t)H > kNoAllocPartialFloats)
+        return fail(ENGRAM_ERR_UNSUPPORTED,
+                    "engram_gate_bwd_noalloc: %lld partial rows x H=%d need %lld floats of scratch, "
+                    "more than its static maximum of %zu",
+                    (long long)G, H, (long long)(G * H), kNoAllocPartialFloats);
+    float *scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != ENGRAM_OK) return st;
+    // Every partial row the reduction reads is written by the backward first
+    // (rows of CTAs without tokens as zeros), so nothing has to be cleared.
+    st = engram_gate_bwd(grad_out, x, k, v, wh, we, T, H, eps, scalar, dx, dk, dv, scratch, G, stream);
+    if (st != ENGRAM_OK) return st;
+    return engram_grad_w_reduce(scratch, G, H, wh, we, dwh, dwe, stream);
+}

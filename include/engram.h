@@ -185,6 +185,36 @@ ENGRAM_API engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t 
                                      engram_stream_t stream);
 
 /*
+ * engram_gate_bwd_noalloc - engram_gate_bwd followed by engram_grad_w_reduce,
+ * allocating nothing, for callers that cannot allocate device memory (code
+ * that may not call cudaMalloc or an allocating library, e.g. under a
+ * capture or memory-pool policy, or a runtime that only owns the buffers it
+ * passes in).  The paper has no counterpart: it is a packaging of the two
+ * calls above.
+ *
+ * Arguments as in engram_gate_bwd, except that the weight-gradient partial
+ * rows are kept in a static device array of the library (8 MiB per GPU that
+ * loads it, held until the process exits) instead of a caller buffer, and the
+ * reduced gradients dwh, dwe (device, fp32 [H], 4-byte aligned, overwritten)
+ * are written directly.  The partial row count is the one
+ * engram_gate_bwd_num_partials(T, H) recommends; if those rows need more than
+ * 2^21 floats the call returns ENGRAM_ERR_UNSUPPORTED and launches nothing.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current): make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents, so calls whose kernels overlap on the GPU (different streams
+ * without ordering between them) race and give wrong gradients; calls in
+ * stream order are fine.  Nothing in the array has to start at zero: every
+ * value the reduction reads is written by the same call first.
+ */
+ENGRAM_API engram_status_t engram_gate_bwd_noalloc(const void *grad_out, const void *x,
+                                        const void *k, const void *v, const void *wh,
+                                        const void *we, int64_t T, int32_t H, float eps,
+                                        float scalar, void *dx, void *dk, void *dv,
+                                        float *dwh, float *dwe, engram_stream_t stream);
+
+/*
  * engram_read_device_error - synchronises the current device, then reads (and
  * when `clear` is non-zero, resets) the device error word in which kernels
  * record a pipeline wait that ran past its time limit.  *code_out receives 0
