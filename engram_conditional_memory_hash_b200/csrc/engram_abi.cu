@@ -75,64 +75,108 @@ engram_status_t device_info(DeviceInfo *out)
 // ------------------------------------------------------------ gate shape ----
 
 constexpr int kGateMaxH = 8192;
-constexpr int kGateMaxStages = 8;
+
+// Launch shape of the gate kernels, chosen by timing launch shapes on B200 at
+// H = 4096 and 7168: the forward runs 2 CTAs per SM of at most 256 threads
+// (4 vectors per thread at H = 7168); the backward, whose registers hold four
+// rows' worth of vectors plus the weight-gradient accumulators, runs one CTA
+// per SM with 2 vectors per thread.  Overridable at compile time.
+#ifndef ENGRAM_FWD_TARGET_THREADS
+#define ENGRAM_FWD_TARGET_THREADS 256
+#endif
+#ifndef ENGRAM_FWD_MAX_CTAS
+#define ENGRAM_FWD_MAX_CTAS 2
+#endif
+#ifndef ENGRAM_BWD_VEC
+#define ENGRAM_BWD_VEC 2
+#endif
+#ifndef ENGRAM_BWD_MAX_CTAS
+#define ENGRAM_BWD_MAX_CTAS 1
+#endif
+#ifndef ENGRAM_GATE_MAX_STAGES
+#define ENGRAM_GATE_MAX_STAGES 8
+#endif
 
 struct GateLaunch {
-    int maxv = 1;       // 16-byte column vectors per thread
+    int maxv = 1;       // 16-byte column vectors per thread (1, 2 or 4)
     int threads = 32;
     int nstage = 2;
     size_t smem = 0;
     int ctas_per_sm = 1;
 };
 
-// Thread count and pipeline depth of a gate kernel streaming `ntensors` rows
-// of H bf16 per token.
-engram_status_t gate_plan(const DeviceInfo &d, int H, int ntensors, GateLaunch *g)
+// Resident CTAs per SM of `kernel` with the given block and shared memory.
+template <typename K>
+engram_status_t occupancy(K kernel, int threads, size_t smem, int *n)
+{
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, kernel, threads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    return ENGRAM_OK;
+}
+
+// Shape of a gate kernel streaming `ntensors` rows of H bf16 per token with
+// `maxv` vectors per thread: the most CTAs per SM (up to max_ctas) that still
+// give each CTA at least two pipeline stages, with as many stages as the
+// shared memory allows.
+template <typename K1, typename K2, typename K4>
+engram_status_t gate_plan(const DeviceInfo &d, int H, int ntensors, int maxv, int max_ctas, K1 k1,
+                          K2 k2, K4 k4, GateLaunch *g)
 {
     const int nvec = H / 8;
-    g->maxv = nvec <= engram::kGateMaxThreads ? 1 : 2;
+    g->maxv = maxv;
     g->threads = ((nvec + g->maxv - 1) / g->maxv + 31) / 32 * 32;
     const size_t stage = (size_t)ntensors * H * 2;
-    const size_t fixed = engram::kGateRedBytes;
-    int ns = (int)(((size_t)d.smem_optin - fixed) / (stage + 8));
-    ns = std::min(ns, kGateMaxStages);
-    if (ns < 2)
-        return fail(ENGRAM_ERR_UNSUPPORTED, "H=%d: two pipeline stages need %zu B of shared memory",
-                    H, 2 * (stage + 8) + fixed);
-    g->nstage = ns;
-    g->smem = engram::gate_smem_bytes(H, ntensors, ns);
-    return ENGRAM_OK;
+    for (int ctas = max_ctas; ctas >= 1; --ctas) {
+        size_t budget = (size_t)d.smem_per_sm / ctas;
+        budget = budget > 1024 ? budget - 1024 : 0;      // per-CTA reserved shared memory
+        budget = std::min(budget, (size_t)d.smem_optin);
+        if (budget <= engram::kGateRedBytes) continue;
+        int ns = (int)((budget - engram::kGateRedBytes) / (stage + 8));
+        ns = std::min(ns, ENGRAM_GATE_MAX_STAGES);
+        if (ns < 2) continue;
+        const size_t smem = engram::gate_smem_bytes(H, ntensors, ns);
+        int n = 0;
+        engram_status_t st = g->maxv == 1 ? occupancy(k1, g->threads, smem, &n)
+                           : g->maxv == 2 ? occupancy(k2, g->threads, smem, &n)
+                                          : occupancy(k4, g->threads, smem, &n);
+        if (st != ENGRAM_OK) return st;
+        if (n < 1) continue;
+        g->nstage = ns;
+        g->smem = smem;
+        g->ctas_per_sm = std::min(n, ctas);
+        return ENGRAM_OK;
+    }
+    return fail(ENGRAM_ERR_UNSUPPORTED, "H=%d: two pipeline stages of %zu B do not fit in shared memory",
+                H, stage);
 }
 
-// Resident CTAs per SM of `kernel` with the plan's block and shared memory.
-template <typename K>
-engram_status_t gate_occupancy(K kernel, GateLaunch *g)
-{
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g->smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-    int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, g->threads, g->smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-    if (n < 1) return fail(ENGRAM_ERR_UNSUPPORTED, "gate kernel does not fit on an SM");
-    g->ctas_per_sm = n;
-    return ENGRAM_OK;
-}
-
-// Forward / backward plan for H, including occupancy.
+// Forward: the fewest vectors per thread that keep the CTA within the target.
 engram_status_t gate_fwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
 {
-    engram_status_t st = gate_plan(d, H, 3, g);
-    if (st != ENGRAM_OK) return st;
-    return g->maxv == 1 ? gate_occupancy(engram::gate_fwd_kernel<1>, g)
-                        : gate_occupancy(engram::gate_fwd_kernel<2>, g);
+    const int nvec = H / 8;
+    int maxv = 4;
+    for (int mv : {1, 2, 4}) {
+        if ((nvec + mv - 1) / mv <= ENGRAM_FWD_TARGET_THREADS) {
+            maxv = mv;
+            break;
+        }
+    }
+    return gate_plan(d, H, 3, maxv, ENGRAM_FWD_MAX_CTAS, engram::gate_fwd_kernel<1>,
+                     engram::gate_fwd_kernel<2>, engram::gate_fwd_kernel<4>, g);
 }
 
+// Backward: ENGRAM_BWD_VEC vectors per thread (one for rows of at most 64
+// vectors, four where two would need more than 512 threads).
 engram_status_t gate_bwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
 {
-    engram_status_t st = gate_plan(d, H, 4, g);
-    if (st != ENGRAM_OK) return st;
-    return g->maxv == 1 ? gate_occupancy(engram::gate_bwd_kernel<1>, g)
-                        : gate_occupancy(engram::gate_bwd_kernel<2>, g);
+    const int nvec = H / 8;
+    int maxv = ENGRAM_BWD_VEC;
+    if (nvec <= 64) maxv = 1;
+    while ((nvec + maxv - 1) / maxv > 1024 / maxv && maxv < 4) maxv *= 2;
+    return gate_plan(d, H, 4, maxv, ENGRAM_BWD_MAX_CTAS, engram::gate_bwd_kernel<1>,
+                     engram::gate_bwd_kernel<2>, engram::gate_bwd_kernel<4>, g);
 }
 
 engram_status_t check_gate_common(int64_t T, int32_t H, float eps, float scalar)
@@ -281,7 +325,9 @@ engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, con
         if (e != cudaSuccess) return cuda_fail(e, "gate_fwd launch");
         return ENGRAM_OK;
     };
-    return g.maxv == 1 ? args(engram::gate_fwd_kernel<1>) : args(engram::gate_fwd_kernel<2>);
+    return g.maxv == 1 ? args(engram::gate_fwd_kernel<1>)
+         : g.maxv == 2 ? args(engram::gate_fwd_kernel<2>)
+                       : args(engram::gate_fwd_kernel<4>);
 }
 
 // ---------------------------------------------------------------- gate bwd ----
@@ -334,7 +380,9 @@ engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void 
         if (e != cudaSuccess) return cuda_fail(e, "gate_bwd launch");
         return ENGRAM_OK;
     };
-    return g.maxv == 1 ? args(engram::gate_bwd_kernel<1>) : args(engram::gate_bwd_kernel<2>);
+    return g.maxv == 1 ? args(engram::gate_bwd_kernel<1>)
+         : g.maxv == 2 ? args(engram::gate_bwd_kernel<2>)
+                       : args(engram::gate_bwd_kernel<4>);
 }
 
 // ----------------------------------------------------------- grad_w_reduce ----
@@ -349,7 +397,8 @@ engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t G, int32_t 
     if (!aligned(w_partial, 4) || !aligned(dwh, 4) || !aligned(dwe, 4) || !aligned(wh, 2) || !aligned(we, 2))
         return fail(ENGRAM_ERR_INVALID_ARG, "misaligned pointer");
     const unsigned blocks = (unsigned)((H + 31) / 32);
-    engram::grad_w_reduce_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+    engram::grad_w_reduce_kernel<<<blocks, engram::kReduceThreads, 0,
+                                   reinterpret_cast<cudaStream_t>(stream)>>>(
         w_partial, G, H, static_cast<const __nv_bfloat16 *>(wh), static_cast<const __nv_bfloat16 *>(we),
         dwh, dwe);
     cudaError_t e = cudaGetLastError();
