@@ -235,37 +235,54 @@ def run_ours(args):
     def to_dev(a):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
 
-    tokens = torch.from_numpy(hin["tokens"]).to(dev)
-    tables = to_dev(hin["tables"])
-    g = {n: to_dev(a) for n, a in gin.items()}
+    tables = torch.from_numpy(hin["tables"].view(np.int16)).view(torch.bfloat16).to(dev)
+    wh = to_dev(gin["wh"])
+    we = to_dev(gin["we"])
     G = eng.engram_gate_bwd_num_partials(T, H)
-    idx = torch.empty((w.B, w.S, L, J), dtype=torch.int64, device=dev)
-    rows = torch.empty((w.B, w.S, L, J, D), dtype=torch.bfloat16, device=dev)
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    gate = torch.empty((T,), dtype=torch.float32, device=dev)
-    dx, dk, dv = (torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(3))
-    part = torch.empty((G, H), dtype=torch.float32, device=dev)
-    dw = torch.empty((2, H), dtype=torch.float32, device=dev)
+
+    def make_buffers(fill: bool):
+        """One set of per-step device buffers (inputs filled from the host when asked)."""
+        b = {"tokens": torch.empty((w.B, w.S), dtype=torch.int64, device=dev)}
+        for n in ("x", "k", "v", "g"):
+            b[n] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        if fill:
+            b["tokens"].copy_(torch.from_numpy(hin["tokens"]))
+            for n in ("x", "k", "v", "g"):
+                b[n].copy_(torch.from_numpy(gin[n].view(np.int16)).view(torch.bfloat16))
+        b["idx"] = torch.empty((w.B, w.S, L, J), dtype=torch.int64, device=dev)
+        b["rows"] = torch.empty((w.B, w.S, L, J, D), dtype=torch.bfloat16, device=dev)
+        b["out"] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        b["gate"] = torch.empty((T,), dtype=torch.float32, device=dev)
+        for n in ("dx", "dk", "dv"):
+            b[n] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        b["part"] = torch.empty((G, H), dtype=torch.float32, device=dev)
+        b["dw"] = torch.empty((2, H), dtype=torch.float32, device=dev)
+        return b
+
+    buf0 = make_buffers(True)
     stream = torch.cuda.current_stream(dev)
     names = ["hash_gather", "gate_fwd", "gate_bwd", "grad_w_reduce"]
 
-    def step(ev=None):
+    def step(b=buf0, ev=None, s=stream):
         def mark(i):
             if ev is not None:
-                ev[i].record(stream)
+                ev[i].record(s)
         mark(0)
-        eng.engram_hash_gather(tokens, hin["multipliers"], hin["ngram_n"], hin["table_sizes"],
-                               tables, pad_id=hin["pad_id"], idx_out=idx, rows_out=rows)
+        eng.engram_hash_gather(b["tokens"], hin["multipliers"], hin["ngram_n"],
+                               hin["table_sizes"], tables, pad_id=hin["pad_id"],
+                               idx_out=b["idx"], rows_out=b["rows"], stream=s)
         mark(1)
-        eng.engram_gate_fwd(g["x"], g["k"], g["v"], g["wh"], g["we"], eps=w.eps, out=out, gate=gate)
+        eng.engram_gate_fwd(b["x"], b["k"], b["v"], wh, we, eps=w.eps, out=b["out"],
+                            gate=b["gate"], stream=s)
         mark(2)
-        eng.engram_gate_bwd(g["g"], g["x"], g["k"], g["v"], g["wh"], g["we"], eps=w.eps,
-                            dx=dx, dk=dk, dv=dv, w_partial=part)
+        eng.engram_gate_bwd(b["g"], b["x"], b["k"], b["v"], wh, we, eps=w.eps, dx=b["dx"],
+                            dk=b["dk"], dv=b["dv"], w_partial=b["part"], stream=s)
         mark(3)
-        eng.engram_grad_w_reduce(part, g["wh"], g["we"], dwh=dw[0], dwe=dw[1])
+        eng.engram_grad_w_reduce(b["part"], wh, we, dwh=b["dw"][0], dwe=b["dw"][1], stream=s)
         mark(4)
         if world > 1:
-            dp.allreduce_weight_grads(dw)
+            with torch.cuda.stream(s):
+                dp.allreduce_weight_grads(b["dw"])
 
     for _ in range(args.warmup):
         step()
@@ -285,7 +302,7 @@ def run_ours(args):
     wall0 = time.time()
     start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step(ev=evs[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
     wall1 = time.time()
@@ -305,6 +322,32 @@ def run_ours(args):
 
     ab = algorithmic_bytes(T, H, L, J, D, G)
     peak, peak_kind = measured_peak()
+
+    # Cache-cold control for the gather: the same hash_gather launch on ids drawn
+    # uniformly over the vocabulary (no hot rows), L2 flushed before each launch.
+    uniform = None
+    if args.uniform_control and rank == 0 and w.vocab > 0:
+        from engram_conditional_memory_hash_b200 import inputs as _inp
+        utok = torch.from_numpy(_inp.uniform_ids(w.seed, 99, (w.B, w.S), 0, w.vocab)).to(dev)
+        flush = torch.empty(2 * 126 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        ts = []
+        for it in range(13):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            eng.engram_hash_gather(utok, hin["multipliers"], hin["ngram_n"], hin["table_sizes"],
+                                   tables, pad_id=hin["pad_id"], idx_out=buf0["idx"],
+                                   rows_out=buf0["rows"], stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= 3:
+                ts.append(e0.elapsed_time(e1))
+        us = float(np.median(ts)) * 1e3
+        gbs = ab["hash_gather"] / (us / 1e6) / 1e9
+        uniform = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
+                   "ids": f"uniform over [0, {w.vocab}), L2 flushed before each launch"}
+        del flush
+
     kern = {}
     for n in names:
         us = per_kernel_ms[n] * 1e3
@@ -328,36 +371,57 @@ def run_ours(args):
     # ---- end to end: host buffers in, host buffers out, copies timed -------
     e2e = None
     if args.e2e_steps > 0:
-        pin = {n: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
-               for n, a in gin.items() if n in ("x", "k", "v", "g")}
-        pin_tok = torch.from_numpy(hin["tokens"]).pin_memory()
-        host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                    for n, t in (("idx", idx), ("rows", rows), ("out", out), ("gate", gate),
-                                 ("dx", dx), ("dk", dk), ("dv", dv), ("dw", dw))}
-        dev_in = {"x": g["x"], "k": g["k"], "v": g["v"], "g": g["g"]}
-        h2d = sum(t.numel() * t.element_size() for t in pin.values()) + pin_tok.numel() * 8
+        # Host buffers in and out: pinned host inputs are uploaded on a copy
+        # stream, the four C-ABI calls run on the compute stream, every output
+        # is downloaded on a second copy stream.  Two device buffer sets let the
+        # upload of step i+1 and the download of step i-1 overlap step i.
+        in_names = ("tokens", "x", "k", "v", "g")
+        out_names = ("idx", "rows", "out", "gate", "dx", "dk", "dv", "dw")
+        host_in = {"tokens": torch.from_numpy(hin["tokens"]).pin_memory()}
+        for n in ("x", "k", "v", "g"):
+            host_in[n] = torch.from_numpy(gin[n].view(np.int16)).view(torch.bfloat16).pin_memory()
+        host_out = {n: torch.empty(buf0[n].shape, dtype=buf0[n].dtype, pin_memory=True)
+                    for n in out_names}
+        bufs = [buf0, make_buffers(False)]
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        comp_s = stream
+        ev_h2d = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_d2h = [torch.cuda.Event() for _ in range(2)]
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-        dev_out = {"idx": idx, "rows": rows, "out": out, "gate": gate, "dx": dx, "dk": dk,
-                   "dv": dv, "dw": dw}
 
-        def e2e_step():
-            tokens.copy_(pin_tok, non_blocking=True)
-            for n, t in pin.items():
-                dev_in[n].copy_(t, non_blocking=True)
-            step()
-            for n, t in host_out.items():
-                t.copy_(dev_out[n], non_blocking=True)
+        def e2e_step(i):
+            bi = i % 2
+            b = bufs[bi]
+            with torch.cuda.stream(h2d_s):
+                if i >= 2:
+                    h2d_s.wait_event(ev_comp[bi])        # inputs of step i-2 consumed
+                for n in in_names:
+                    b[n].copy_(host_in[n], non_blocking=True)
+                ev_h2d[bi].record(h2d_s)
+            comp_s.wait_event(ev_h2d[bi])
+            if i >= 2:
+                comp_s.wait_event(ev_d2h[bi])            # outputs of step i-2 downloaded
+            step(b, s=comp_s)
+            ev_comp[bi].record(comp_s)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(ev_comp[bi])
+                for n in out_names:
+                    host_out[n].copy_(b[n], non_blocking=True)
+                ev_d2h[bi].record(d2h_s)
 
-        e2e_step()
+        for i in range(2):                                # warm-up
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         s0 = torch.cuda.Event(enable_timing=True)
         s1 = torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        s1.record(stream)
+        s0.record(h2d_s)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        s1.record(d2h_s)
         torch.cuda.synchronize(dev)
         e_ms = s0.elapsed_time(s1)
         if world > 1:
@@ -367,7 +431,9 @@ def run_ours(args):
         e2e = {"value": round(world * T / (e_ms / args.e2e_steps / 1e3), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps,
-               "path": "pinned host inputs -> H2D -> C-ABI calls -> D2H of every output"}
+               "path": "pinned host inputs -> H2D (copy stream) -> the four C-ABI calls -> D2H "
+                       "of every output (second copy stream); two device buffer sets overlap "
+                       "step i's compute with the neighbouring steps' copies"}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) -------
     cpu = None
@@ -411,6 +477,7 @@ def run_ours(args):
                 world * T / ((per_kernel_ms["gate_fwd"] + per_kernel_ms["gate_bwd"]
                               + per_kernel_ms["grad_w_reduce"]) / 1e3), 1),
             "kernels": kern,
+            "hash_gather_uniform_ids": uniform,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -474,9 +541,11 @@ def main():
     ap.add_argument("--workload", default="full_path")
     ap.add_argument("--tokens", type=int, default=0,
                     help="cut the workload to its first N tokens (profiling runs)")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-uniform-control", dest="uniform_control", action="store_false",
+                    help="skip the uniform-id hash_gather control measurement")
     ap.add_argument("--ref-tokens", type=int, default=32)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

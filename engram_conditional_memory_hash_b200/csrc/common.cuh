@@ -28,22 +28,24 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&p);
 }
 
-// 8 bf16 values of a 16-byte vector -> 8 floats.
-__device__ __forceinline__ void unpack8(const uint4 &q, float f[8])
+// 8 bf16 values of a 16-byte vector -> 4 float pairs (element 2i in .x).
+__device__ __forceinline__ void unpack4x2(const uint4 &q, float2 f[4])
 {
-    f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x);
-    f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
-    f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z);
-    f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
+    f[0] = make_float2(bf16_lo(q.x), bf16_hi(q.x));
+    f[1] = make_float2(bf16_lo(q.y), bf16_hi(q.y));
+    f[2] = make_float2(bf16_lo(q.z), bf16_hi(q.z));
+    f[3] = make_float2(bf16_lo(q.w), bf16_hi(q.w));
 }
 
-__device__ __forceinline__ uint4 pack8(const float f[8])
+__device__ __forceinline__ uint32_t pack_bf16x2(float2 f) { return pack_bf16(f.x, f.y); }
+
+__device__ __forceinline__ uint4 pack4x2(const float2 f[4])
 {
     uint4 q;
-    q.x = pack_bf16(f[0], f[1]);
-    q.y = pack_bf16(f[2], f[3]);
-    q.z = pack_bf16(f[4], f[5]);
-    q.w = pack_bf16(f[6], f[7]);
+    q.x = pack_bf16x2(f[0]);
+    q.y = pack_bf16x2(f[1]);
+    q.z = pack_bf16x2(f[2]);
+    q.w = pack_bf16x2(f[3]);
     return q;
 }
 

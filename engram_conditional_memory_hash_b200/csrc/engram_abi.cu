@@ -158,7 +158,8 @@ engram_status_t gate_fwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
     const int nvec = H / 8;
     int maxv = 4;
     for (int mv : {1, 2, 4}) {
-        if ((nvec + mv - 1) / mv <= ENGRAM_FWD_TARGET_THREADS) {
+        const int t = (nvec + mv - 1) / mv;
+        if (t <= ENGRAM_FWD_TARGET_THREADS && t <= engram::gate_max_threads(mv)) {
             maxv = mv;
             break;
         }
@@ -174,7 +175,7 @@ engram_status_t gate_bwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
     const int nvec = H / 8;
     int maxv = ENGRAM_BWD_VEC;
     if (nvec <= 64) maxv = 1;
-    while ((nvec + maxv - 1) / maxv > 1024 / maxv && maxv < 4) maxv *= 2;
+    while ((nvec + maxv - 1) / maxv > engram::gate_max_threads(maxv) && maxv < 4) maxv *= 2;
     return gate_plan(d, H, 4, maxv, ENGRAM_BWD_MAX_CTAS, engram::gate_bwd_kernel<1>,
                      engram::gate_bwd_kernel<2>, engram::gate_bwd_kernel<4>, g);
 }

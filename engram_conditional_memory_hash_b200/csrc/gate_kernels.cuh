@@ -36,9 +36,10 @@
 
 namespace engram {
 
-// Largest CTA of a gate kernel whose threads own MAXV column vectors each.
-template <int MAXV>
-constexpr int gate_max_threads() { return 1024 / MAXV; }
+// Largest CTA of a gate kernel whose threads own `maxv` column vectors each
+// (rows of up to 8192 values; one vector per thread caps the CTA at 512 so
+// that those threads may hold 128 registers).
+__host__ __device__ constexpr int gate_max_threads(int maxv) { return maxv == 1 ? 512 : 1024 / maxv; }
 // Block reduction: per warp and token parity, the fp32 sums (float4) and the
 // fp64 dot product (double).
 constexpr size_t kGateRedBytes = 2 * 32 * sizeof(float4) + 2 * 32 * sizeof(double);
@@ -51,6 +52,14 @@ __host__ __device__ inline size_t gate_smem_bytes(int H, int ntensors, int nstag
            + (size_t)nstage * 8u;                             // one mbarrier per stage
 }
 
+// Extra bytes added to every stage's expected transaction count.  Always 0 in
+// the library; the pipeline-timeout test builds a copy of the library with a
+// non-zero value, so that no stage ever completes and every wait runs into
+// its time limit (nothing faults: the copies themselves are unchanged).
+#ifndef ENGRAM_TEST_EXTRA_TX
+#define ENGRAM_TEST_EXTRA_TX 0u
+#endif
+
 // Issue the bulk copies of token `row` (NTENSORS rows of row_bytes) into stage
 // `s`.  Called by one thread.
 template <int NTENSORS>
@@ -61,7 +70,7 @@ __device__ __forceinline__ void gate_issue_row(unsigned char *smem, uint32_t bar
     const uint32_t stage_bytes = NTENSORS * row_bytes;
     const uint32_t dst = smem_addr(smem + (size_t)s * stage_bytes);
     const uint32_t bar = bar0 + 8u * (uint32_t)s;
-    mbar_arrive_expect_tx(bar, stage_bytes);
+    mbar_arrive_expect_tx(bar, stage_bytes + ENGRAM_TEST_EXTRA_TX);
 #pragma unroll
     for (int q = 0; q < NTENSORS; ++q) {
         const char *p = static_cast<const char *>(src[q]) + row * (int64_t)row_bytes;
@@ -110,6 +119,37 @@ __device__ __forceinline__ void gate_pipeline_start(unsigned char *smem, uint32_
     }
 }
 
+#ifndef ENGRAM_COMBINE_SHUFFLE
+#define ENGRAM_COMBINE_SHUFFLE 0
+#endif
+
+// Sum of the per-warp partials of one token, in a fixed order: every thread
+// either adds the nwarps entries in warp order, or (ENGRAM_COMBINE_SHUFFLE)
+// lane q takes warp q's entry and a shuffle tree adds them.
+__device__ __forceinline__ void combine_partials(const float4 *rb, const double *rbd, int nwarps,
+                                                 int lane, float4 &r, double &A)
+{
+#if ENGRAM_COMBINE_SHUFFLE
+    r = lane < nwarps ? rb[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+    A = lane < nwarps ? rbd[lane] : 0.0;
+    r.x = warp_sum(r.x);
+    r.y = warp_sum(r.y);
+    r.z = warp_sum(r.z);
+    A = warp_sum_f64(A);
+#else
+    (void)lane;
+    r = make_float4(0.f, 0.f, 0.f, 0.f);
+    A = 0.0;
+    for (int q = 0; q < nwarps; ++q) {
+        const float4 t = rb[q];
+        r.x += t.x;
+        r.y += t.y;
+        r.z += t.z;
+        A += rbd[q];
+    }
+#endif
+}
+
 // Per-token gate from the reduced statistics.
 struct GateScalars {
     float rx, rk, d, s, gate;
@@ -132,7 +172,7 @@ __device__ __forceinline__ GateScalars gate_scalars(float Sx, float Sk, double A
 // --------------------------------------------------------------- forward ----
 
 template <int MAXV>
-__global__ void __launch_bounds__(gate_max_threads<MAXV>(), MAXV == 4 ? 2 : 1)
+__global__ void __launch_bounds__(gate_max_threads(MAXV), MAXV == 4 ? 2 : 1)
 gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
                 const uint4 *__restrict__ v, const uint4 *__restrict__ wh,
                 const uint4 *__restrict__ we, int64_t T, int H, float eps, float scalar,
@@ -155,16 +195,20 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
 #pragma unroll
     for (int m = 0; m < MAXV; ++m) {
         const int vi = tid + m * nthreads;
-        float a[8], b[8];
+        float2 a[4], b[4];
         if (vi < nvec) {
-            unpack8(wh[vi], a);
-            unpack8(we[vi], b);
+            unpack4x2(wh[vi], a);
+            unpack4x2(we[vi], b);
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = b[e] = 0.f;
+            for (int e = 0; e < 4; ++e) a[e] = b[e] = make_float2(0.f, 0.f);
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) w[m][e] = (double)(a[e] * b[e]);
+        for (int e = 0; e < 4; ++e) {
+            const float2 p = __fmul2_rn(a[e], b[e]);
+            w[m][2 * e] = (double)p.x;
+            w[m][2 * e + 1] = (double)p.y;
+        }
     }
 
     const int64_t G = gridDim.x, first = blockIdx.x;
@@ -181,7 +225,7 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
         const uint4 *sv = sk + nvec;
 
         uint4 xq[MAXV], vq[MAXV];
-        float px = 0.f, pk = 0.f;
+        float2 px2 = make_float2(0.f, 0.f), pk2 = px2;
         double pa = 0.0;
 #pragma unroll
         for (int m = 0; m < MAXV; ++m) {
@@ -189,19 +233,21 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
             if (vi < nvec) {
                 xq[m] = sx[vi];
                 vq[m] = sv[vi];
-                float xf[8], kf[8];
-                unpack8(xq[m], xf);
-                unpack8(sk[vi], kf);
+                float2 xf[4], kf[4];
+                unpack4x2(xq[m], xf);
+                unpack4x2(sk[vi], kf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    px = fmaf(xf[e], xf[e], px);
-                    pk = fmaf(kf[e], kf[e], pk);
-                    pa = fma((double)(xf[e] * kf[e]), w[m][e], pa);
+                for (int e = 0; e < 4; ++e) {
+                    px2 = __ffma2_rn(xf[e], xf[e], px2);
+                    pk2 = __ffma2_rn(kf[e], kf[e], pk2);
+                    const float2 xk = __fmul2_rn(xf[e], kf[e]);   // exact
+                    pa = fma((double)xk.x, w[m][2 * e], pa);
+                    pa = fma((double)xk.y, w[m][2 * e + 1], pa);
                 }
             }
         }
-        px = warp_sum(px);
-        pk = warp_sum(pk);
+        float px = warp_sum(px2.x + px2.y);
+        float pk = warp_sum(pk2.x + pk2.y);
         pa = warp_sum_f64(pa);
         float4 *rb = red + (i & 1) * 32;
         double *rbd = redd + (i & 1) * 32;
@@ -221,28 +267,24 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
         if (tid == 0 && i + nstage < nrows)
             gate_issue_row<3>(smem, bar0, src, first + (i + nstage) * G, row_bytes, s);
 
-        float Sx = 0.f, Sk = 0.f;
-        double A = 0.0;
-        for (int q = 0; q < nwarps; ++q) {
-            const float4 r = rb[q];
-            Sx += r.x;
-            Sk += r.y;
-            A += rbd[q];
-        }
-        const GateScalars c = gate_scalars(Sx, Sk, A, inv_h, eps, scalar);
+        float4 r;
+        double A;
+        combine_partials(rb, rbd, nwarps, lane, r, A);
+        const GateScalars c = gate_scalars(r.x, r.y, A, inv_h, eps, scalar);
 
         const int64_t row = first + i * G;
         uint4 *orow = out + row * nvec;
+        const float2 gate2 = make_float2(c.gate, c.gate);
 #pragma unroll
         for (int m = 0; m < MAXV; ++m) {
             const int vi = tid + m * nthreads;
             if (vi < nvec) {
-                float xf[8], vf[8], of[8];
-                unpack8(xq[m], xf);
-                unpack8(vq[m], vf);
+                float2 xf[4], vf[4], of[4];
+                unpack4x2(xq[m], xf);
+                unpack4x2(vq[m], vf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) of[e] = fmaf(c.gate, vf[e], xf[e]);
-                __stcs(orow + vi, pack8(of));
+                for (int e = 0; e < 4; ++e) of[e] = __ffma2_rn(gate2, vf[e], xf[e]);
+                __stcs(orow + vi, pack4x2(of));
             }
         }
         if (tid == 0 && gate != nullptr) gate[row] = c.gate;
@@ -252,7 +294,7 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
 // -------------------------------------------------------------- backward ----
 
 template <int MAXV>
-__global__ void __launch_bounds__(gate_max_threads<MAXV>(), 1)
+__global__ void __launch_bounds__(gate_max_threads(MAXV), 1)
 gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
                 const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                 const uint4 *__restrict__ wh, const uint4 *__restrict__ we, int64_t T, int H,
@@ -271,22 +313,22 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nthreads = blockDim.x, nwarps = nthreads >> 5;
 
-    float w[MAXV][8], acc[MAXV][8];
+    float2 w[MAXV][4], acc[MAXV][4];
 #pragma unroll
     for (int m = 0; m < MAXV; ++m) {
         const int vi = tid + m * nthreads;
         if (vi < nvec) {
-            float a[8], b[8];
-            unpack8(wh[vi], a);
-            unpack8(we[vi], b);
+            float2 a[4], b[4];
+            unpack4x2(wh[vi], a);
+            unpack4x2(we[vi], b);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w[m][e] = a[e] * b[e];
+            for (int e = 0; e < 4; ++e) w[m][e] = __fmul2_rn(a[e], b[e]);
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w[m][e] = 0.f;
+            for (int e = 0; e < 4; ++e) w[m][e] = make_float2(0.f, 0.f);
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[m][e] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[m][e] = make_float2(0.f, 0.f);
     }
 
     const int64_t G = gridDim.x, first = blockIdx.x;
@@ -304,7 +346,7 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
         const uint4 *sv = sk + nvec;
 
         uint4 gq[MAXV], xq[MAXV], kq[MAXV];
-        float px = 0.f, pk = 0.f, pg = 0.f;
+        float2 px2 = make_float2(0.f, 0.f), pk2 = px2, pg2 = px2;
         double pa = 0.0;
 #pragma unroll
         for (int m = 0; m < MAXV; ++m) {
@@ -313,24 +355,26 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
                 gq[m] = sg[vi];
                 xq[m] = sx[vi];
                 kq[m] = sk[vi];
-                float gf[8], xf[8], kf[8], vf[8];
-                unpack8(gq[m], gf);
-                unpack8(xq[m], xf);
-                unpack8(kq[m], kf);
-                unpack8(sv[vi], vf);
+                float2 gf[4], xf[4], kf[4], vf[4];
+                unpack4x2(gq[m], gf);
+                unpack4x2(xq[m], xf);
+                unpack4x2(kq[m], kf);
+                unpack4x2(sv[vi], vf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    px = fmaf(xf[e], xf[e], px);
-                    pk = fmaf(kf[e], kf[e], pk);
-                    pa = fma((double)(xf[e] * kf[e]), (double)w[m][e], pa);
-                    pg = fmaf(gf[e], vf[e], pg);
+                for (int e = 0; e < 4; ++e) {
+                    px2 = __ffma2_rn(xf[e], xf[e], px2);
+                    pk2 = __ffma2_rn(kf[e], kf[e], pk2);
+                    pg2 = __ffma2_rn(gf[e], vf[e], pg2);
+                    const float2 xk = __fmul2_rn(xf[e], kf[e]);   // exact
+                    pa = fma((double)xk.x, (double)w[m][e].x, pa);
+                    pa = fma((double)xk.y, (double)w[m][e].y, pa);
                 }
             }
         }
-        px = warp_sum(px);
-        pk = warp_sum(pk);
+        float px = warp_sum(px2.x + px2.y);
+        float pk = warp_sum(pk2.x + pk2.y);
+        float pg = warp_sum(pg2.x + pg2.y);
         pa = warp_sum_f64(pa);
-        pg = warp_sum(pg);
         float4 *rb = red + (i & 1) * 32;
         double *rbd = redd + (i & 1) * 32;
         if (lane == 0) {
@@ -347,16 +391,11 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
         if (tid == 0 && i + nstage < nrows)
             gate_issue_row<4>(smem, bar0, src, first + (i + nstage) * G, row_bytes, s);
 
-        float Sx = 0.f, Sk = 0.f, Sg = 0.f;
-        double A = 0.0;
-        for (int q = 0; q < nwarps; ++q) {
-            const float4 r = rb[q];
-            Sx += r.x;
-            Sk += r.y;
-            Sg += r.z;
-            A += rbd[q];
-        }
-        const GateScalars c = gate_scalars(Sx, Sk, A, inv_h, eps, scalar);
+        float4 r;
+        double A;
+        combine_partials(rb, rbd, nwarps, lane, r, A);
+        const float Sg = r.z;
+        const GateScalars c = gate_scalars(r.x, r.y, A, inv_h, eps, scalar);
         // chain rule through sigmoid, signed_sqrt (|s| clamped at 1e-6), scalar
         const float du = Sg * c.gate * (1.0f - c.gate);
         const float dd = du * 0.5f * rsqrtf(fmaxf(fabsf(c.s), 1e-6f)) * scalar;
@@ -368,25 +407,27 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
         uint4 *dxr = dx + row * nvec;
         uint4 *dkr = dk + row * nvec;
         uint4 *dvr = dv + row * nvec;
+        const float2 c1v = make_float2(c1, c1), nc2 = make_float2(-c2, -c2);
+        const float2 nc3 = make_float2(-c3, -c3), gate2 = make_float2(c.gate, c.gate);
 #pragma unroll
         for (int m = 0; m < MAXV; ++m) {
             const int vi = tid + m * nthreads;
             if (vi < nvec) {
-                float gf[8], xf[8], kf[8], a[8], b[8], cv[8];
-                unpack8(gq[m], gf);
-                unpack8(xq[m], xf);
-                unpack8(kq[m], kf);
+                float2 gf[4], xf[4], kf[4], a[4], b[4], cv[4];
+                unpack4x2(gq[m], gf);
+                unpack4x2(xq[m], xf);
+                unpack4x2(kq[m], kf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float cw = c1 * w[m][e];
-                    a[e] = fmaf(-c2, xf[e], fmaf(cw, kf[e], gf[e]));
-                    b[e] = fmaf(-c3, kf[e], cw * xf[e]);
-                    cv[e] = c.gate * gf[e];
-                    acc[m][e] = fmaf(c1, xf[e] * kf[e], acc[m][e]);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 cw = __fmul2_rn(c1v, w[m][e]);
+                    a[e] = __ffma2_rn(nc2, xf[e], __ffma2_rn(cw, kf[e], gf[e]));
+                    b[e] = __ffma2_rn(nc3, kf[e], __fmul2_rn(cw, xf[e]));
+                    cv[e] = __fmul2_rn(gate2, gf[e]);
+                    acc[m][e] = __ffma2_rn(c1v, __fmul2_rn(xf[e], kf[e]), acc[m][e]);
                 }
-                __stcs(dxr + vi, pack8(a));
-                __stcs(dkr + vi, pack8(b));
-                __stcs(dvr + vi, pack8(cv));
+                __stcs(dxr + vi, pack4x2(a));
+                __stcs(dkr + vi, pack4x2(b));
+                __stcs(dvr + vi, pack4x2(cv));
             }
         }
     }
@@ -397,8 +438,8 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
     for (int m = 0; m < MAXV; ++m) {
         const int vi = tid + m * nthreads;
         if (vi < nvec) {
-            prow[2 * vi] = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
-            prow[2 * vi + 1] = make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]);
+            prow[2 * vi] = make_float4(acc[m][0].x, acc[m][0].y, acc[m][1].x, acc[m][1].y);
+            prow[2 * vi + 1] = make_float4(acc[m][2].x, acc[m][2].y, acc[m][3].x, acc[m][3].y);
         }
     }
 }
