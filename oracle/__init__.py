@@ -71,6 +71,9 @@ class Oracle:
         lib.oracle_engram_gate_bwd.argtypes = [
             _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int64, ctypes.c_int32,
             ctypes.c_double, ctypes.c_double, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p]
+        lib.oracle_engram_gather_bwd.argtypes = [
+            _i64p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _i64p, _f64p, ctypes.c_int32,
+            ctypes.c_int64, ctypes.c_int64, _f64p]
         self.lib = lib
         self.path = lib_path
 
@@ -127,6 +130,32 @@ class Oracle:
         out = np.empty((T, L, J, D), dtype=np.uint16)
         self.lib.oracle_engram_gather(ip, T, L, J, tsp, tabp, D, out.ctypes.data_as(_u16p))
         return out.reshape(*lead, L, J, D)
+
+    def engram_gather_bwd(self, idx, table_sizes, d_rows, row_lo: int = 0, row_hi=None):
+        """Transpose of the gather: d_rows [..., L, J, D] (float64, or bf16 bits as
+        uint16) summed into the table rows they were read from.  Returns the
+        global rows [row_lo, row_hi) of the concatenated tables, [rows, D] float64."""
+        ts, tsp = _c(table_sizes, np.int64, _i64p)
+        L, J = ts.shape
+        if L * J > 256:
+            raise ValueError("the oracle supports at most 256 tables")
+        idx = np.asarray(idx)
+        idx2, ip = _c(idx.reshape(-1, L, J), np.int64, _i64p)
+        if np.any(idx2 < 0) or np.any(idx2 >= ts[None, :, :]):
+            raise ValueError("index out of range")
+        T = idx2.shape[0]
+        dr = _widen(d_rows)
+        D = dr.shape[-1]
+        dr = np.ascontiguousarray(dr.reshape(T, L, J, D))
+        R = int(ts.sum())
+        if row_hi is None:
+            row_hi = R
+        if not 0 <= row_lo <= row_hi <= R:
+            raise ValueError("bad row range")
+        out = np.empty((row_hi - row_lo, D), dtype=np.float64)
+        self.lib.oracle_engram_gather_bwd(ip, T, L, J, tsp, dr.ctypes.data_as(_f64p), D,
+                                          int(row_lo), int(row_hi), out.ctypes.data_as(_f64p))
+        return out
 
     def engram_gate_fwd(self, x, k, v, wh, we, eps: float = 1e-6, scalar: float | None = None):
         """Gate forward.  x, k, v [T, H]; wh, we [H].
@@ -209,6 +238,10 @@ def engram_hash(*a, **kw):
 
 def engram_gather(*a, **kw):
     return default().engram_gather(*a, **kw)
+
+
+def engram_gather_bwd(*a, **kw):
+    return default().engram_gather_bwd(*a, **kw)
 
 
 def engram_gate_fwd(*a, **kw):

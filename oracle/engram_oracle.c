@@ -95,6 +95,16 @@ void oracle_engram_hash(const int64_t *tokens, int64_t B, int64_t S,
     }
 }
 
+/* First row of each table in the concatenated tables (at most 256 tables). */
+static void table_first_rows(const int64_t *table_sizes, int32_t ntab, int64_t *first_row)
+{
+    int64_t acc = 0;
+    for (int32_t q = 0; q < ntab && q < 256; ++q) {
+        first_row[q] = acc;
+        acc += table_sizes[q];
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Table-row gather.  tables holds the L*J tables one after another, table  */
 /* (l,j) with table_sizes[l*J+j] rows of D bf16 values.  rows_out[T*L*J*D]  */
@@ -106,11 +116,7 @@ void oracle_engram_gather(const int64_t *idx, int64_t T, int32_t L, int32_t J,
 {
     int32_t ntab = L * J;
     int64_t first_row[256];
-    int64_t acc = 0;
-    for (int32_t q = 0; q < ntab && q < 256; ++q) {
-        first_row[q] = acc;
-        acc += table_sizes[q];
-    }
+    table_first_rows(table_sizes, ntab, first_row);
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         for (int32_t q = 0; q < ntab; ++q) {
@@ -265,6 +271,36 @@ void oracle_engram_gate_bwd(const double *grad_out, const double *x,
         for (int32_t j = j0; j < j1; ++j) {
             dwh[j] = sh[j - j0];
             dwe[j] = se[j - j0];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Gather backward: the gradient reaching a gathered row is added to the     */
+/* table row it was read from, so a row read several times receives the sum */
+/* of their gradients (the transpose of the gather above).                   */
+/* idx [T*L*J] local rows as from oracle_engram_hash; d_rows [T*L*J*D];      */
+/* d_tables receives the global rows [row_lo, row_hi) of the concatenated    */
+/* tables, (row_hi - row_lo) * D doubles, overwritten:                       */
+/*   d_tables[r - row_lo][c] = sum over (t, l, j) with                      */
+/*        first_row(l, j) + idx[t][l][j] == r  of  d_rows[t][l][j][c],      */
+/* summed in (t, l, j) order.                                                */
+/* ------------------------------------------------------------------------ */
+void oracle_engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int32_t J,
+                              const int64_t *table_sizes, const double *d_rows, int32_t D,
+                              int64_t row_lo, int64_t row_hi, double *d_tables)
+{
+    int32_t ntab = L * J;
+    int64_t first_row[256];
+    table_first_rows(table_sizes, ntab, first_row);
+    for (int64_t i = 0; i < (row_hi - row_lo) * D; ++i) d_tables[i] = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t q = 0; q < ntab; ++q) {
+            int64_t r = first_row[q] + idx[t * ntab + q];
+            if (r < row_lo || r >= row_hi) continue;
+            const double *src = d_rows + (t * ntab + q) * D;
+            double *dst = d_tables + (r - row_lo) * D;
+            for (int32_t c = 0; c < D; ++c) dst[c] += src[c];
         }
     }
 }

@@ -132,6 +132,48 @@ def pin_gather_rows(o):
 
 
 # --------------------------------------------------------------------------
+# gather backward (the transpose of the gather)
+# --------------------------------------------------------------------------
+
+def pin_gather_bwd_handworked(o):
+    # one layer, two tables of 3 and 2 rows (global rows 0-2 and 3-4), D = 2
+    idx = np.array([[[0, 1]], [[2, 1]], [[0, 0]]], dtype=np.int64).reshape(3, 1, 2)
+    sizes = np.array([[3, 2]], dtype=np.int64)
+    d_rows = np.arange(1, 13, dtype=np.float64).reshape(3, 1, 2, 2)
+    got = o.engram_gather_bwd(idx, sizes, d_rows)
+    # row 0 <- tokens 0 and 2 of table 0; row 2 <- token 1; row 3 <- token 2 of
+    # table 1; row 4 <- tokens 0 and 1 of table 1; row 1 is never read
+    want = np.array([[1 + 9, 2 + 10], [0, 0], [5, 6], [11, 12], [3 + 7, 4 + 8]], dtype=np.float64)
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal(o.engram_gather_bwd(idx, sizes, d_rows, 2, 4), want[2:4])
+
+
+def pin_gather_bwd_adjoint_and_conservation(o):
+    # <gather(y), d> = <y, gather_bwd(d)> for any table values y and gradients d,
+    # and the gradient mass is conserved column by column
+    w = inputs.WORKLOADS["tiny"]
+    h = inputs.hash_inputs(w, with_tables=False)
+    P = h["table_sizes"]
+    idx = o.engram_hash(h["tokens"], h["multipliers"], h["ngram_n"], P, pad_id=h["pad_id"])
+    r = np.random.default_rng(17)
+    D = 8
+    R = int(P.sum())
+    y = r.standard_normal((R, D))
+    d = r.standard_normal(idx.shape + (D,))
+    first = np.concatenate([[0], np.cumsum(P.ravel())[:-1]]).reshape(1, 1, 2, 8)
+    gathered = y[idx + first]
+    g = o.engram_gather_bwd(idx, P, d)
+    assert g.shape == (R, D)
+    lhs = float((gathered * d).sum())
+    rhs = float((y * g).sum())
+    assert abs(lhs - rhs) <= 1e-9 * max(1.0, abs(lhs)), (lhs, rhs)
+    np.testing.assert_allclose(g.sum(0), d.reshape(-1, D).sum(0), rtol=1e-12, atol=1e-10)
+    untouched = np.ones(R, dtype=bool)
+    untouched[(idx + first).ravel()] = False
+    assert np.all(g[untouched] == 0.0)
+
+
+# --------------------------------------------------------------------------
 # gate forward
 # --------------------------------------------------------------------------
 
@@ -321,7 +363,8 @@ def pin_thread_count_independent(o):
 
 
 HASH_PINS = [pin_hash_handworked, pin_hash_unsigned_modulo, pin_hash_wrapping_multiply,
-             pin_hash_bruteforce, pin_hash_invariants, pin_gather_rows]
+             pin_hash_bruteforce, pin_hash_invariants, pin_gather_rows,
+             pin_gather_bwd_handworked, pin_gather_bwd_adjoint_and_conservation]
 GATE_PINS = [pin_fwd_orthogonal_gives_half, pin_fwd_v_zero_is_identity,
              pin_fwd_parallel_closed_form, pin_fwd_eps_enters_rms, pin_fwd_scale_invariance,
              pin_bwd_finite_differences, pin_bwd_matches_autograd, pin_bwd_clamp_at_zero,
