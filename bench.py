@@ -39,6 +39,7 @@ METRIC = "Engram gate fwd+bwd tokens/s and HBM GB/s (% of B200 peak) at H=7168"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["engram_conditional_memory_hash_b200/csrc/gate_kernels.cuh",
                   "engram_conditional_memory_hash_b200/csrc/hash_gather.cuh",
+                  "engram_conditional_memory_hash_b200/csrc/gather_bwd.cuh",
                   "engram_conditional_memory_hash_b200/csrc/common.cuh",
                   "engram_conditional_memory_hash_b200/csrc/engram_abi.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -348,6 +349,44 @@ def run_ours(args):
                    "ids": f"uniform over [0, {w.vocab}), L2 flushed before each launch"}
         del flush
 
+    # Gather backward (the transpose of the gather: row gradients summed into
+    # the fp32 table gradient), timed on its own: it is not one of the four
+    # calls of the step.  d_rows is a synthetic N(0,1) gradient of the gathered
+    # rows; d_tables (4.1 GB) accumulates across iterations, which does not
+    # change the work.
+    gbwd = None
+    if args.gather_bwd and rank == 0 and w.has_hash:
+        from engram_conditional_memory_hash_b200 import inputs as _inp
+        d_rows = torch.from_numpy(_inp.gather_grad_inputs(w).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        R = int(hin["table_sizes"].sum())
+        d_tables = torch.zeros((R, D), dtype=torch.float32, device=dev)
+        ws = torch.empty((eng.engram_gather_bwd_workspace_size(T, L, J, D),), dtype=torch.uint8,
+                         device=dev)
+        first = torch.from_numpy(np.concatenate(
+            [[0], np.cumsum(hin["table_sizes"].ravel())[:-1]])).to(dev)
+        uniq = int(torch.unique(buf0["idx"].view(T, L * J) + first[None]).numel())
+        ts = []
+        for it in range(13):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            eng.engram_gather_bwd(buf0["idx"], hin["table_sizes"], d_rows, d_tables, workspace=ws,
+                                  stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= 3:
+                ts.append(e0.elapsed_time(e1))
+        us = float(np.median(ts)) * 1e3
+        # idx read + d_rows read + one read and one write of every touched fp32 table row
+        gb_bytes = T * L * J * (8 + 2 * D) + uniq * 2 * 4 * D
+        gbs = gb_bytes / (us / 1e6) / 1e9
+        gbwd = {"us": round(us, 2), "algorithmic_bytes": gb_bytes, "GB/s": round(gbs, 1),
+                "frac": round(gbs / peak, 4), "unique_rows": uniq, "entries": T * L * J,
+                "launches": 11,
+                "what": "engram_gather_bwd on the step's indices: radix sort of (row, entry), "
+                        "segmented fp64 sums, fp32 table-gradient update; median of 10 calls"}
+        del d_rows, d_tables, ws
+
     kern = {}
     for n in names:
         us = per_kernel_ms[n] * 1e3
@@ -478,6 +517,7 @@ def run_ours(args):
                               + per_kernel_ms["grad_w_reduce"]) / 1e3), 1),
             "kernels": kern,
             "hash_gather_uniform_ids": uniform,
+            "gather_bwd": gbwd,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -546,6 +586,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-uniform-control", dest="uniform_control", action="store_false",
                     help="skip the uniform-id hash_gather control measurement")
+    ap.add_argument("--no-gather-bwd", dest="gather_bwd", action="store_false",
+                    help="skip the separate engram_gather_bwd measurement")
     ap.add_argument("--ref-tokens", type=int, default=32)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

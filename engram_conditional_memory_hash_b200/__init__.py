@@ -1,8 +1,9 @@
 """Engram conditional-memory hot path for NVIDIA B200 (sm_100a).
 
 Thin Python binding of the C-ABI library ``libengram_b200.so`` (declared in
-``include/engram.h``): the n-gram hash with its table-row gather, and the
-fused Engram gate forward/backward with the weight-gradient reduction, as
+``include/engram.h``): the n-gram hash with its table-row gather and the
+gather's backward into the tables, and the fused Engram gate
+forward/backward with the weight-gradient reduction, as
 listed on the page "DeepSeek 开源 TileKernels" (zhichai.net/topic/177618722),
 section "5. Engram — 条件记忆门控".
 
@@ -27,7 +28,8 @@ __all__ = [
     "EngramError", "library_path", "lib", "engram_abi_version",
     "engram_hash_gather", "engram_gate_fwd", "engram_gate_bwd_num_partials",
     "engram_gate_bwd", "engram_grad_w_reduce", "engram_read_device_error",
-    "engram_gate_bwd_noalloc", "default_scalar",
+    "engram_gate_bwd_noalloc", "engram_gather_bwd_workspace_size", "engram_gather_bwd",
+    "default_scalar", "DEVICE_ERR_PIPELINE_TIMEOUT", "DEVICE_ERR_INDEX_RANGE",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +37,11 @@ LIBRARY_NAME = "libengram_b200.so"
 EXPORTED = ("engram_abi_version", "engram_status_string", "engram_last_error",
             "engram_hash_gather", "engram_gate_fwd", "engram_gate_bwd_num_partials",
             "engram_gate_bwd", "engram_grad_w_reduce", "engram_read_device_error",
-            "engram_gate_bwd_noalloc")
+            "engram_gate_bwd_noalloc", "engram_gather_bwd_workspace_size", "engram_gather_bwd")
+
+# codes of the kernels' device error word (engram_read_device_error)
+DEVICE_ERR_PIPELINE_TIMEOUT = 1
+DEVICE_ERR_INDEX_RANGE = 2
 
 
 class EngramError(RuntimeError):
@@ -92,6 +98,11 @@ def lib() -> ctypes.CDLL:
             L.engram_gate_bwd_noalloc.restype = ctypes.c_int
             L.engram_gate_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _f32,
                                                   _f32, _vp, _vp, _vp, _vp, _vp, _vp]
+            L.engram_gather_bwd_workspace_size.restype = _i64
+            L.engram_gather_bwd_workspace_size.argtypes = [_i64, _i32, _i32, _i32]
+            L.engram_gather_bwd.restype = ctypes.c_int
+            L.engram_gather_bwd.argtypes = [_vp, _i64, _i32, _i32, _vp, _vp, _i32, _vp, _vp,
+                                            ctypes.c_size_t, _vp]
             L.engram_read_device_error.restype = ctypes.c_int
             L.engram_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), _i32]
             _lib = L
@@ -190,6 +201,59 @@ def engram_hash_gather(tokens: torch.Tensor, multipliers, ngram_n, table_sizes,
                                   _stream_ptr(stream))
     _check("engram_hash_gather", st)
     return (idx_out if want_idx else None), (rows_out if want_rows else None)
+
+
+def engram_gather_bwd_workspace_size(T: int, L: int, J: int, D: int) -> int:
+    """Bytes of device workspace engram_gather_bwd needs (raises for sizes it rejects)."""
+    n = int(lib().engram_gather_bwd_workspace_size(int(T), int(L), int(J), int(D)))
+    if n < 0:
+        _check("engram_gather_bwd_workspace_size", 2)
+    return n
+
+
+def engram_gather_bwd(idx: torch.Tensor, table_sizes, d_rows: torch.Tensor,
+                      d_tables: torch.Tensor | None = None, *,
+                      workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Backward of the row gather: d_tables[row of (t, l, j)] += d_rows[t, l, j].
+
+    idx          int64 [..., L, J] on the GPU (as returned by engram_hash_gather).
+    table_sizes  host [L, J].
+    d_rows       bf16 [..., L, J, D] on the GPU, the gradient of the gathered rows
+                 (one row per entry of idx, in the same order).
+    d_tables     fp32 [sum(table_sizes), D] on the GPU, accumulated in place
+                 (a zero tensor is allocated when None).
+    workspace    uint8 tensor of at least engram_gather_bwd_workspace_size bytes
+                 (allocated when None).
+    Returns d_tables.
+    """
+    ts = _host(table_sizes, np.int64)
+    if ts.ndim != 2:
+        raise ValueError("table_sizes must be [L, J]")
+    L, J = ts.shape
+    ip = _dev(idx, "idx", torch.int64)
+    rp = _dev(d_rows, "d_rows", torch.bfloat16)
+    if idx.dim() < 2 or tuple(idx.shape[-2:]) != (L, J):
+        raise ValueError("idx must be [..., L, J]")
+    T = idx.numel() // (L * J)
+    if d_rows.dim() < 3 or tuple(d_rows.shape[-3:-1]) != (L, J):
+        raise ValueError("d_rows must be [..., L, J, D]")
+    D = d_rows.shape[-1]
+    if d_rows.numel() != T * L * J * D:
+        raise ValueError("d_rows must hold one row per entry of idx")
+    R = int(ts.sum())
+    if d_tables is None:
+        d_tables = torch.zeros((R, D), dtype=torch.float32, device=d_rows.device)
+    tp = _dev(d_tables, "d_tables", torch.float32)
+    if tuple(d_tables.shape) != (R, D):
+        raise ValueError("d_tables must be [sum(table_sizes), D]")
+    need = engram_gather_bwd_workspace_size(T, L, J, D)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=d_rows.device)
+    wp = _dev(workspace, "workspace", torch.uint8)
+    st = lib().engram_gather_bwd(ip, T, L, J, ts.ctypes.data, rp, D, tp, wp, workspace.numel(),
+                                 _stream_ptr(stream))
+    _check("engram_gather_bwd", st)
+    return d_tables
 
 
 # ----------------------------------------------------------------- gate ----

@@ -16,6 +16,7 @@
 
 #include "common.cuh"
 #include "gate_kernels.cuh"
+#include "gather_bwd.cuh"
 #include "hash_gather.cuh"
 
 namespace {
@@ -188,6 +189,54 @@ engram_status_t check_gate_common(int64_t T, int32_t H, float eps, float scalar)
         return fail(ENGRAM_ERR_UNSUPPORTED, "H=%d: must be a multiple of 8 in [8, %d]", H, kGateMaxH);
     if (!std::isfinite(eps) || eps < 0.f) return fail(ENGRAM_ERR_INVALID_ARG, "eps must be finite and >= 0");
     if (!std::isfinite(scalar)) return fail(ENGRAM_ERR_INVALID_ARG, "scalar must be finite");
+    return ENGRAM_OK;
+}
+
+// ------------------------------------------------------- gather backward ----
+
+constexpr int64_t kGbwdMaxEntries = int64_t(1) << 30;
+
+// Offsets (bytes, 256-aligned) of the gather backward's scratch in the
+// caller's workspace: two (key, position) buffers for the radix passes, the
+// digit histograms, and the fp64 partial rows of chunk-crossing segments.
+struct GbwdLayout {
+    int64_t ntiles = 0, nchunks = 0, nhist = 0;
+    size_t keys_a = 0, vals_a = 0, keys_b = 0, vals_b = 0, hist = 0, carry_a = 0, carry_b = 0;
+    size_t total = 0;
+};
+
+GbwdLayout gbwd_layout(int64_t N, int D)
+{
+    GbwdLayout g;
+    g.ntiles = (N + engram::kSortTile - 1) / engram::kSortTile;
+    g.nchunks = (N + engram::kSegChunk - 1) / engram::kSegChunk;
+    g.nhist = (int64_t)engram::kRadixBins * g.ntiles;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + 255) & ~size_t(255);
+        return o;
+    };
+    g.keys_a = take((size_t)N * 4);
+    g.vals_a = take((size_t)N * 4);
+    g.keys_b = take((size_t)N * 4);
+    g.vals_b = take((size_t)N * 4);
+    g.hist = take((size_t)g.nhist * 4);
+    g.carry_a = take((size_t)g.nchunks * (size_t)D * 8);
+    g.carry_b = take((size_t)g.nchunks * (size_t)D * 8);
+    g.total = off;
+    return g;
+}
+
+engram_status_t check_gbwd_sizes(int64_t T, int32_t L, int32_t J, int32_t D)
+{
+    if (T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
+    if (L < 1 || L > engram::kHashMaxL) return fail(ENGRAM_ERR_UNSUPPORTED, "L=%d not in [1, %d]", L, engram::kHashMaxL);
+    if (J < 1 || J > engram::kHashMaxJ) return fail(ENGRAM_ERR_UNSUPPORTED, "J=%d not in [1, %d]", J, engram::kHashMaxJ);
+    if (D < 8 || D > 256 || D % 8 != 0)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "D=%d: must be a multiple of 8 in [8, 256]", D);
+    if (T > kGbwdMaxEntries / (L * J))
+        return fail(ENGRAM_ERR_UNSUPPORTED, "T*L*J above 2^30 entries");
     return ENGRAM_OK;
 }
 
@@ -407,6 +456,102 @@ engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t G, int32_t 
     return ENGRAM_OK;
 }
 
+// -------------------------------------------------------- gather backward ----
+
+int64_t engram_gather_bwd_workspace_size(int64_t T, int32_t L, int32_t J, int32_t D)
+{
+    if (check_gbwd_sizes(T, L, J, D) != ENGRAM_OK) return -1;
+    return (int64_t)gbwd_layout(T * L * J, D).total;
+}
+
+engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int32_t J,
+                                  const int64_t *table_sizes, const void *d_rows, int32_t D,
+                                  float *d_tables, void *workspace, size_t workspace_bytes,
+                                  engram_stream_t stream)
+{
+    using engram::GatherBwdParams;
+    engram_status_t st = check_gbwd_sizes(T, L, J, D);
+    if (st != ENGRAM_OK) return st;
+    if (!table_sizes) return fail(ENGRAM_ERR_INVALID_ARG, "table_sizes is required");
+    GatherBwdParams p;
+    std::memset(&p, 0, sizeof p);
+    p.LJ = L * J;
+    p.D = D;
+    int64_t R = 0;
+    for (int q = 0; q < p.LJ; ++q) {
+        const int64_t P = table_sizes[q];
+        if (P < 1) return fail(ENGRAM_ERR_INVALID_ARG, "table_sizes[%d]=%lld < 1", q, (long long)P);
+        if (P > int64_t(0xfffffffe) - R)
+            return fail(ENGRAM_ERR_UNSUPPORTED, "total table rows must stay below 2^32 - 1");
+        p.P[q] = (uint32_t)P;
+        p.row0[q] = (uint32_t)R;
+        R += P;
+    }
+    p.R = (uint32_t)R;
+    const int64_t N = T * p.LJ;
+    p.N = N;
+    if (N == 0) return ENGRAM_OK;
+    if (!idx || !d_rows || !d_tables || !workspace)
+        return fail(ENGRAM_ERR_INVALID_ARG, "idx, d_rows, d_tables and workspace are required");
+    if (!aligned(idx, 8)) return fail(ENGRAM_ERR_INVALID_ARG, "idx must be 8-byte aligned");
+    if (!aligned(d_rows, 16) || !aligned(d_tables, 16) || !aligned(workspace, 16))
+        return fail(ENGRAM_ERR_INVALID_ARG, "d_rows, d_tables and workspace must be 16-byte aligned");
+    const GbwdLayout g = gbwd_layout(N, D);
+    if (workspace_bytes < g.total)
+        return fail(ENGRAM_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, g.total);
+
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    uint32_t *keys[2] = {reinterpret_cast<uint32_t *>(ws + g.keys_a), reinterpret_cast<uint32_t *>(ws + g.keys_b)};
+    uint32_t *vals[2] = {reinterpret_cast<uint32_t *>(ws + g.vals_a), reinterpret_cast<uint32_t *>(ws + g.vals_b)};
+    uint32_t *hist = reinterpret_cast<uint32_t *>(ws + g.hist);
+    double2 *carry_a = reinterpret_cast<double2 *>(ws + g.carry_a);
+    double2 *carry_b = reinterpret_cast<double2 *>(ws + g.carry_b);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    // keys lie in [0, R] (R marks an invalid entry): sort on their bit length
+    int nbits = 0;
+    while (nbits < 32 && (uint64_t(R) >> nbits) != 0) ++nbits;
+    const int npasses = (nbits + 7) / 8;
+    const unsigned ntiles = (unsigned)g.ntiles;
+    int cur = 0;
+    for (int pass = 0; pass < npasses; ++pass) {
+        const int shift = 8 * pass;
+        const int dst = pass == 0 ? 0 : 1 - cur;
+        if (pass == 0) {
+            engram::gbwd_hist_kernel<true><<<ntiles, engram::kSortThreads, 0, s>>>(idx, nullptr, p, shift, hist);
+        } else {
+            engram::gbwd_hist_kernel<false><<<ntiles, engram::kSortThreads, 0, s>>>(nullptr, keys[cur], p, shift, hist);
+        }
+        engram::gbwd_scan_kernel<<<1, engram::kScanThreads, 0, s>>>(hist, g.nhist);
+        if (pass == 0) {
+            engram::gbwd_scatter_kernel<true><<<ntiles, engram::kSortThreads, 0, s>>>(
+                idx, nullptr, nullptr, p, shift, hist, keys[dst], vals[dst]);
+        } else {
+            engram::gbwd_scatter_kernel<false><<<ntiles, engram::kSortThreads, 0, s>>>(
+                nullptr, keys[cur], vals[cur], p, shift, hist, keys[dst], vals[dst]);
+        }
+        cur = dst;
+    }
+    const int64_t seg_blocks = (g.nchunks + engram::kSegThreads / 32 - 1) / (engram::kSegThreads / 32);
+    const unsigned blocks = (unsigned)std::min<int64_t>(seg_blocks, int64_t(1) << 30);
+    const __nv_bfloat162 *rows = static_cast<const __nv_bfloat162 *>(d_rows);
+    float2 *tab = reinterpret_cast<float2 *>(d_tables);
+    const int npairs = D / 2;
+    if (npairs <= 32) {
+        engram::gbwd_segment_kernel<1><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], vals[cur], rows, p, tab, carry_a, carry_b);
+        engram::gbwd_carry_kernel<1><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], p, tab, carry_a, carry_b);
+    } else if (npairs <= 64) {
+        engram::gbwd_segment_kernel<2><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], vals[cur], rows, p, tab, carry_a, carry_b);
+        engram::gbwd_carry_kernel<2><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], p, tab, carry_a, carry_b);
+    } else {
+        engram::gbwd_segment_kernel<4><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], vals[cur], rows, p, tab, carry_a, carry_b);
+        engram::gbwd_carry_kernel<4><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], p, tab, carry_a, carry_b);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "gather_bwd launch");
+    return ENGRAM_OK;
+}
+
 // ------------------------------------------------------------ diagnostics ----
 
 engram_status_t engram_read_device_error(uint32_t *code_out, int32_t clear)
@@ -432,8 +577,8 @@ engram_status_t engram_read_device_error(uint32_t *code_out, int32_t clear)
 //
 // engram_gate_bwd_noalloc: engram_gate_bwd followed by engram_grad_w_reduce
 // for callers that cannot allocate device memory (for example code running
-// under a memory-pool or graph-capture policy that forbids cudaMalloc, or a
-// host runtime whose only device buffers are the ones it was handed).  The
+// under a memory-pool policy that forbids cudaMalloc, or a host runtime whose
+// only device buffers are the ones it was handed).  The
 // weight-gradient partial rows, the only scratch of the backward, live in the
 // fixed array below instead of a caller-provided buffer.
 

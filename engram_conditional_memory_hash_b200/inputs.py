@@ -17,6 +17,8 @@ on the number of host threads):
 * table sizes: ``count`` consecutive primes from ``base`` upward, assigned to
   tables in (layer, table) order.
 * tables: bf16 N(0,1), all tables concatenated row-major.
+* d_rows (the gradient reaching the gathered rows, for the gather backward):
+  bf16 N(0,1) of shape [T, L, J, D].
 
 The workloads (token count T = B*S, hidden size H, tables of D columns):
 
@@ -45,6 +47,7 @@ CHUNK = 1 << 22  # elements per independently seeded chunk
 STREAM_X, STREAM_K, STREAM_V, STREAM_G = 0, 1, 2, 3
 STREAM_WH, STREAM_WE = 4, 5
 STREAM_TOKENS, STREAM_MULT, STREAM_TABLES = 6, 7, 8
+STREAM_DROWS = 9
 
 
 def generator(seed: int, *stream: int) -> np.random.Generator:
@@ -208,3 +211,9 @@ def hash_inputs(w: Workload, B: int | None = None, S: int | None = None,
         rows = int(out["table_sizes"].sum())
         out["tables"] = normal_bf16(w.seed, STREAM_TABLES, (rows, w.D))
     return out
+
+
+def gather_grad_inputs(w: Workload, T: int | None = None) -> np.ndarray:
+    """d_rows [T, L, J, D] as bf16 bits (uint16): the gradient of the gathered rows."""
+    T = w.T if T is None else T
+    return normal_bf16(w.seed, STREAM_DROWS, (T, w.L, w.J, w.D))

@@ -59,6 +59,7 @@ typedef enum {
 
 /* Codes a kernel may record in the device error word. */
 #define ENGRAM_DEVICE_ERR_PIPELINE_TIMEOUT 1u
+#define ENGRAM_DEVICE_ERR_INDEX_RANGE 2u   /* engram_gather_bwd met an index outside its table */
 
 /* Version of this ABI (incremented on any incompatible change). */
 ENGRAM_API int engram_abi_version(void);
@@ -108,6 +109,54 @@ ENGRAM_API engram_status_t engram_hash_gather(const int64_t *tokens, int64_t B, 
                                    int32_t L, int32_t n_max, const int64_t *table_sizes,
                                    int32_t J, const void *tables, int32_t D, int64_t pad_id,
                                    int64_t *idx_out, void *rows_out, engram_stream_t stream);
+
+/*
+ * engram_gather_bwd_workspace_size - bytes of device workspace that
+ * engram_gather_bwd needs for T tokens, L layers, J tables per layer and rows
+ * of D values.  Returns -1 (with engram_last_error() set) for sizes that
+ * engram_gather_bwd rejects.  No device is queried.
+ */
+ENGRAM_API int64_t engram_gather_bwd_workspace_size(int64_t T, int32_t L, int32_t J, int32_t D);
+
+/*
+ * engram_gather_bwd - backward of the row gather of engram_hash_gather with
+ * respect to the tables.  The page above lists only the gather; its gradient
+ * is the transpose of a row copy: every gathered row's gradient is added to
+ * the table row it was read from, so a row read by several tokens receives
+ * the sum of their gradients:
+ *     d_tables[row0(l,j) + idx[t][l][j]][c] += d_rows[t][l][j][c]
+ * with row0(l,j) the first row of table (l, j) in the concatenated tables.
+ * Rows that no token read are left untouched (d_tables accumulates, like a
+ * parameter gradient: zero it before the first call of a step).
+ *
+ * The gradients of one row are summed in fp64 (bf16 values enter exactly) in
+ * an order fixed by the positions of the entries, and the row is updated with
+ * one rounding: d_tables[r] = fp32((double)d_tables[r] + sum).  The result is
+ * bitwise reproducible.
+ *
+ * idx         device, int64 [T*L*J] laid out [t][l][j] (as written by
+ *             engram_hash_gather), 8-byte aligned; each entry must lie in
+ *             [0, table_sizes[l*J + j]).  An entry outside that range is
+ *             skipped and the kernels record ENGRAM_DEVICE_ERR_INDEX_RANGE
+ *             (see engram_read_device_error); nothing outside the buffers is
+ *             touched.
+ * T           >= 0 tokens (0 launches nothing; the pointers may then be NULL).
+ * L, J        1..4 layers, 1..16 tables per layer; T*L*J <= 2^30.
+ * table_sizes HOST, int64 [L*J], each >= 1, total rows R below 2^32 - 1.
+ * d_rows      device, bf16 [T*L*J*D] laid out [t][l][j][D], 16-byte aligned:
+ *             the gradient of the gathered rows.
+ * D           row width: a multiple of 8, 8..256.
+ * d_tables    device, fp32 [R*D], row-major, 16-byte aligned; accumulated.
+ * workspace   device scratch of at least workspace_bytes >=
+ *             engram_gather_bwd_workspace_size(T, L, J, D) bytes, 16-byte
+ *             aligned, owned by the caller; its contents need not be
+ *             initialised and are meaningless afterwards.  Calls in flight at
+ *             the same time need separate workspaces.
+ */
+ENGRAM_API engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int32_t J,
+                                  const int64_t *table_sizes, const void *d_rows, int32_t D,
+                                  float *d_tables, void *workspace, size_t workspace_bytes,
+                                  engram_stream_t stream);
 
 /*
  * engram_gate_fwd - fused Engram gate forward ("engram_gate_fwd" on the page
@@ -187,9 +236,9 @@ ENGRAM_API engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t 
 /*
  * engram_gate_bwd_noalloc - engram_gate_bwd followed by engram_grad_w_reduce,
  * allocating nothing, for callers that cannot allocate device memory (code
- * that may not call cudaMalloc or an allocating library, e.g. under a
- * capture or memory-pool policy, or a runtime that only owns the buffers it
- * passes in).  The paper has no counterpart: it is a packaging of the two
+ * that may not call cudaMalloc or an allocating library, e.g. a runtime whose
+ * memory policy forbids allocations outside its own pool, or one that only
+ * owns the buffers it passes in).  The paper has no counterpart: it is a packaging of the two
  * calls above.
  *
  * Arguments as in engram_gate_bwd, except that the weight-gradient partial

@@ -128,3 +128,44 @@ def test_python_binding_rejects_cpu_tensors():
 def test_no_device_is_reported_not_hidden():
     assert eng.lib().engram_gate_bwd_num_partials(1024, 4096) == -1
     assert eng.lib().engram_last_error()
+
+
+def test_gather_bwd_rejects_before_launch():
+    import numpy as np
+    L = eng.lib()
+    ts = np.full((2, 8), 4099, dtype=np.int64)
+    p = ctypes.c_void_p(64)
+
+    def gb(T=4, L_=2, J=8, ts=ts, D=32, idx=p, rows=p, tab=p, ws=p, nbytes=1 << 30):
+        return L.engram_gather_bwd(idx, T, L_, J, ts.ctypes.data if ts is not None else None,
+                                   rows, D, tab, ws, nbytes, None)
+
+    assert gb(T=-1) == INVALID
+    assert gb(L_=0) == UNSUPPORTED and gb(L_=5) == UNSUPPORTED
+    assert gb(J=0) == UNSUPPORTED and gb(J=17) == UNSUPPORTED
+    assert gb(D=12) == UNSUPPORTED and gb(D=264) == UNSUPPORTED
+    assert gb(T=2**27) == UNSUPPORTED                                  # 2^31 entries
+    assert gb(ts=None) == INVALID
+    bad = ts.copy()
+    bad[0, 2] = 0
+    assert gb(ts=bad) == INVALID
+    big = np.full((2, 8), 2**28, dtype=np.int64)                       # 2^32 rows in total
+    assert gb(ts=big) == UNSUPPORTED
+    assert gb(idx=None) == INVALID and gb(ws=None) == INVALID
+    assert gb(idx=ctypes.c_void_p(68)) == INVALID                      # idx not 8-aligned
+    assert gb(rows=ctypes.c_void_p(72)) == INVALID                     # d_rows not 16-aligned
+    assert gb(tab=ctypes.c_void_p(72)) == INVALID
+    assert gb(nbytes=16) == INVALID                                    # workspace too small
+    assert b"workspace" in L.engram_last_error()
+    assert gb(T=0, idx=None, rows=None, tab=None, ws=None) == OK       # empty: nothing to launch
+
+
+def test_gather_bwd_workspace_size():
+    # two (key, position) arrays of 4-byte words per radix pass, the digit
+    # histograms and two fp64 partial rows per chunk of 64 sorted entries
+    n = eng.engram_gather_bwd_workspace_size(65536, 2, 8, 64)
+    N = 65536 * 16
+    assert 16 * N <= n <= 16 * N + 256 * (N // 4096) * 4 + 2 * (N // 64) * 64 * 8 + 8 * 256
+    assert eng.engram_gather_bwd_workspace_size(0, 2, 8, 64) == 0
+    with pytest.raises(eng.EngramError):
+        eng.engram_gather_bwd_workspace_size(4, 2, 8, 12)
