@@ -126,6 +126,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     return true;
 }
 
+// Programmatic dependent launch (sm_90 and later).  Wait until the kernel
+// that precedes this one in the stream has completed and its writes are
+// visible (a no-op when the launch carries no programmatic dependency), then
+// let the next kernel of the stream be scheduled: it in turn waits here for
+// this whole grid to complete before it reads anything, so the early release
+// only overlaps launch latency with this kernel's tail.
+__device__ __forceinline__ void pdl_wait_and_release()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void record_device_error(unsigned code)
 {
     atomicOr(&g_device_error, code);

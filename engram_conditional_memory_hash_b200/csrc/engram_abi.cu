@@ -194,14 +194,37 @@ engram_status_t check_gate_common(int64_t T, int32_t H, float eps, float scalar)
 
 // ------------------------------------------------------- gather backward ----
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel of the stream drains; every kernel launched this
+// way starts with pdl_wait_and_release(), so it reads nothing before its
+// predecessor has completed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t s,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr int64_t kGbwdMaxEntries = int64_t(1) << 30;
 
 // Offsets (bytes, 256-aligned) of the gather backward's scratch in the
 // caller's workspace: two (key, position) buffers for the radix passes, the
-// digit histograms, and the fp64 partial rows of chunk-crossing segments.
+// digit histograms and digit totals, and the fp64 partial rows of
+// chunk-crossing segments with the list of chunks where such segments end.
 struct GbwdLayout {
     int64_t ntiles = 0, nchunks = 0, nhist = 0;
-    size_t keys_a = 0, vals_a = 0, keys_b = 0, vals_b = 0, hist = 0, carry_a = 0, carry_b = 0;
+    size_t keys_a = 0, vals_a = 0, keys_b = 0, vals_b = 0, hist = 0, totals = 0, carry_a = 0,
+           carry_b = 0, carry_list = 0, carry_count = 0;
     size_t total = 0;
 };
 
@@ -222,9 +245,12 @@ GbwdLayout gbwd_layout(int64_t N, int D)
     g.keys_b = take((size_t)N * 4);
     g.vals_b = take((size_t)N * 4);
     g.hist = take((size_t)g.nhist * 4);
+    g.totals = take((size_t)engram::kRadixBins * 4);
     g.carry_a = take((size_t)g.nchunks * (size_t)D * 8);
     g.carry_b = take((size_t)g.nchunks * (size_t)D * 8);
-    g.total = off;
+    g.carry_list = take((size_t)g.nchunks * 4);
+    g.carry_count = take(4);
+    g.total = N > 0 ? off : 0;
     return g;
 }
 
@@ -461,7 +487,7 @@ engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t G, int32_t 
 int64_t engram_gather_bwd_workspace_size(int64_t T, int32_t L, int32_t J, int32_t D)
 {
     if (check_gbwd_sizes(T, L, J, D) != ENGRAM_OK) return -1;
-    return (int64_t)gbwd_layout(T * L * J, D).total;
+    return (int64_t)gbwd_layout(T * L * J, D).total;   // 0 when T == 0
 }
 
 engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int32_t J,
@@ -504,50 +530,73 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     uint32_t *keys[2] = {reinterpret_cast<uint32_t *>(ws + g.keys_a), reinterpret_cast<uint32_t *>(ws + g.keys_b)};
     uint32_t *vals[2] = {reinterpret_cast<uint32_t *>(ws + g.vals_a), reinterpret_cast<uint32_t *>(ws + g.vals_b)};
     uint32_t *hist = reinterpret_cast<uint32_t *>(ws + g.hist);
-    double2 *carry_a = reinterpret_cast<double2 *>(ws + g.carry_a);
-    double2 *carry_b = reinterpret_cast<double2 *>(ws + g.carry_b);
+    uint32_t *totals = reinterpret_cast<uint32_t *>(ws + g.totals);
+    double *carry_a = reinterpret_cast<double *>(ws + g.carry_a);
+    double *carry_b = reinterpret_cast<double *>(ws + g.carry_b);
+    uint32_t *carry_list = reinterpret_cast<uint32_t *>(ws + g.carry_list);
+    uint32_t *carry_count = reinterpret_cast<uint32_t *>(ws + g.carry_count);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t *no_idx = nullptr;
+    const uint32_t *no_u32 = nullptr;
+    uint32_t *no_count = nullptr;
 
     // keys lie in [0, R] (R marks an invalid entry): sort on their bit length
     int nbits = 0;
     while (nbits < 32 && (uint64_t(R) >> nbits) != 0) ++nbits;
     const int npasses = (nbits + 7) / 8;
     const unsigned ntiles = (unsigned)g.ntiles;
+    const unsigned T_ = engram::kSortThreads;
+    cudaError_t e = cudaSuccess;
     int cur = 0;
-    for (int pass = 0; pass < npasses; ++pass) {
+    for (int pass = 0; pass < npasses && e == cudaSuccess; ++pass) {
         const int shift = 8 * pass;
         const int dst = pass == 0 ? 0 : 1 - cur;
-        if (pass == 0) {
-            engram::gbwd_hist_kernel<true><<<ntiles, engram::kSortThreads, 0, s>>>(idx, nullptr, p, shift, hist);
-        } else {
-            engram::gbwd_hist_kernel<false><<<ntiles, engram::kSortThreads, 0, s>>>(nullptr, keys[cur], p, shift, hist);
-        }
-        engram::gbwd_scan_kernel<<<1, engram::kScanThreads, 0, s>>>(hist, g.nhist);
-        if (pass == 0) {
-            engram::gbwd_scatter_kernel<true><<<ntiles, engram::kSortThreads, 0, s>>>(
-                idx, nullptr, nullptr, p, shift, hist, keys[dst], vals[dst]);
-        } else {
-            engram::gbwd_scatter_kernel<false><<<ntiles, engram::kSortThreads, 0, s>>>(
-                nullptr, keys[cur], vals[cur], p, shift, hist, keys[dst], vals[dst]);
+        if (pass == 0)
+            e = launch_pdl(engram::gbwd_hist_kernel<true>, ntiles, T_, s, idx, no_u32, p, shift, hist, carry_count);
+        else
+            e = launch_pdl(engram::gbwd_hist_kernel<false>, ntiles, T_, s, no_idx, keys[cur], p, shift, hist, no_count);
+        if (e == cudaSuccess)
+            e = launch_pdl(engram::gbwd_digit_scan_kernel, (unsigned)engram::kRadixBins,
+                           (unsigned)engram::kScanThreads, s, hist, g.ntiles, totals);
+        if (e == cudaSuccess) {
+            if (pass == 0)
+                e = launch_pdl(engram::gbwd_scatter_kernel<true>, ntiles, T_, s, idx, no_u32, no_u32, p,
+                               shift, hist, totals, keys[dst], vals[dst]);
+            else
+                e = launch_pdl(engram::gbwd_scatter_kernel<false>, ntiles, T_, s, no_idx, keys[cur], vals[cur],
+                               p, shift, hist, totals, keys[dst], vals[dst]);
         }
         cur = dst;
     }
     const int64_t seg_blocks = (g.nchunks + engram::kSegThreads / 32 - 1) / (engram::kSegThreads / 32);
     const unsigned blocks = (unsigned)std::min<int64_t>(seg_blocks, int64_t(1) << 30);
-    const __nv_bfloat162 *rows = static_cast<const __nv_bfloat162 *>(d_rows);
-    float2 *tab = reinterpret_cast<float2 *>(d_tables);
-    const int npairs = D / 2;
-    if (npairs <= 32) {
-        engram::gbwd_segment_kernel<1><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], vals[cur], rows, p, tab, carry_a, carry_b);
-        engram::gbwd_carry_kernel<1><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], p, tab, carry_a, carry_b);
-    } else if (npairs <= 64) {
-        engram::gbwd_segment_kernel<2><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], vals[cur], rows, p, tab, carry_a, carry_b);
-        engram::gbwd_carry_kernel<2><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], p, tab, carry_a, carry_b);
-    } else {
-        engram::gbwd_segment_kernel<4><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], vals[cur], rows, p, tab, carry_a, carry_b);
-        engram::gbwd_carry_kernel<4><<<blocks, engram::kSegThreads, 0, s>>>(keys[cur], p, tab, carry_a, carry_b);
+    const uint4 *rows = static_cast<const uint4 *>(d_rows);
+    float4 *tab4 = reinterpret_cast<float4 *>(d_tables);
+    const unsigned S_ = engram::kSegThreads;
+    const int nv = D / 8;   // 16-byte vectors per row: lanes per segment group
+    if (e == cudaSuccess) {
+        if (nv <= 4)
+            e = launch_pdl(engram::gbwd_segment_kernel<4, 2>, blocks, S_, s, keys[cur], vals[cur], rows, p,
+                           tab4, carry_a, carry_b, carry_list, carry_count);
+        else if (nv <= 8)
+            e = launch_pdl(engram::gbwd_segment_kernel<8, 2>, blocks, S_, s, keys[cur], vals[cur], rows, p,
+                           tab4, carry_a, carry_b, carry_list, carry_count);
+        else if (nv <= 16)
+            e = launch_pdl(engram::gbwd_segment_kernel<16, 2>, blocks, S_, s, keys[cur], vals[cur], rows, p,
+                           tab4, carry_a, carry_b, carry_list, carry_count);
+        else
+            e = launch_pdl(engram::gbwd_segment_kernel<32, 2>, blocks, S_, s, keys[cur], vals[cur], rows, p,
+                           tab4, carry_a, carry_b, carry_list, carry_count);
     }
-    cudaError_t e = cudaGetLastError();
+    // one warp per listed chunk (a warp loops when more than 4096 are listed)
+    const int64_t carry_warps = std::min<int64_t>(g.nchunks, 4096);
+    const unsigned carry_blocks = (unsigned)((carry_warps + engram::kCarryThreads / 32 - 1) /
+                                             (engram::kCarryThreads / 32));
+    if (e == cudaSuccess)
+        e = launch_pdl(engram::gbwd_carry_kernel, carry_blocks, (unsigned)engram::kCarryThreads, s,
+                       static_cast<const uint32_t *>(keys[cur]), p, d_tables,
+                       static_cast<const double *>(carry_a), static_cast<const double *>(carry_b),
+                       static_cast<const uint32_t *>(carry_list), static_cast<const uint32_t *>(carry_count));
     if (e != cudaSuccess) return cuda_fail(e, "gather_bwd launch");
     return ENGRAM_OK;
 }
