@@ -99,7 +99,7 @@ def lib() -> ctypes.CDLL:
             L.engram_gate_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _f32,
                                                   _f32, _vp, _vp, _vp, _vp, _vp, _vp]
             L.engram_gather_bwd_workspace_size.restype = _i64
-            L.engram_gather_bwd_workspace_size.argtypes = [_i64, _i32, _i32, _i32]
+            L.engram_gather_bwd_workspace_size.argtypes = [_i64, _i32, _i32, _i32, _i64]
             L.engram_gather_bwd.restype = ctypes.c_int
             L.engram_gather_bwd.argtypes = [_vp, _i64, _i32, _i32, _vp, _vp, _i32, _vp, _vp,
                                             ctypes.c_size_t, _vp]
@@ -203,9 +203,11 @@ def engram_hash_gather(tokens: torch.Tensor, multipliers, ngram_n, table_sizes,
     return (idx_out if want_idx else None), (rows_out if want_rows else None)
 
 
-def engram_gather_bwd_workspace_size(T: int, L: int, J: int, D: int) -> int:
-    """Bytes of device workspace engram_gather_bwd needs (raises for sizes it rejects)."""
-    n = int(lib().engram_gather_bwd_workspace_size(int(T), int(L), int(J), int(D)))
+def engram_gather_bwd_workspace_size(T: int, L: int, J: int, D: int, total_rows: int) -> int:
+    """Bytes of device workspace engram_gather_bwd needs for T tokens, L x J tables of
+    total_rows rows of D values (raises for sizes it rejects)."""
+    n = int(lib().engram_gather_bwd_workspace_size(int(T), int(L), int(J), int(D),
+                                                   int(total_rows)))
     if n < 0:
         _check("engram_gather_bwd_workspace_size", 2)
     return n
@@ -246,7 +248,7 @@ def engram_gather_bwd(idx: torch.Tensor, table_sizes, d_rows: torch.Tensor,
     tp = _dev(d_tables, "d_tables", torch.float32)
     if tuple(d_tables.shape) != (R, D):
         raise ValueError("d_tables must be [sum(table_sizes), D]")
-    need = engram_gather_bwd_workspace_size(T, L, J, D)
+    need = engram_gather_bwd_workspace_size(T, L, J, D, R)
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=d_rows.device)
     wp = _dev(workspace, "workspace", torch.uint8)

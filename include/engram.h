@@ -112,11 +112,14 @@ ENGRAM_API engram_status_t engram_hash_gather(const int64_t *tokens, int64_t B, 
 
 /*
  * engram_gather_bwd_workspace_size - bytes of device workspace that
- * engram_gather_bwd needs for T tokens, L layers, J tables per layer and rows
- * of D values.  Returns -1 (with engram_last_error() set) for sizes that
- * engram_gather_bwd rejects.  No device is queried.
+ * engram_gather_bwd needs for T tokens, L layers, J tables per layer, rows of
+ * D values and total_rows rows in all tables together (the sum of
+ * table_sizes).  About 32 bytes per entry plus 2 bits per table row.  Returns
+ * -1 (with engram_last_error() set) for sizes that engram_gather_bwd rejects.
+ * No device is queried.
  */
-ENGRAM_API int64_t engram_gather_bwd_workspace_size(int64_t T, int32_t L, int32_t J, int32_t D);
+ENGRAM_API int64_t engram_gather_bwd_workspace_size(int64_t T, int32_t L, int32_t J, int32_t D,
+                                                    int64_t total_rows);
 
 /*
  * engram_gather_bwd - backward of the row gather of engram_hash_gather with
@@ -148,7 +151,7 @@ ENGRAM_API int64_t engram_gather_bwd_workspace_size(int64_t T, int32_t L, int32_
  * D           row width: a multiple of 8, 8..256.
  * d_tables    device, fp32 [R*D], row-major, 16-byte aligned; accumulated.
  * workspace   device scratch of at least workspace_bytes >=
- *             engram_gather_bwd_workspace_size(T, L, J, D) bytes, 16-byte
+ *             engram_gather_bwd_workspace_size(T, L, J, D, R) bytes, 16-byte
  *             aligned, owned by the caller; its contents need not be
  *             initialised and are meaningless afterwards.  Calls in flight at
  *             the same time need separate workspaces.

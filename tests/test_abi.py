@@ -161,13 +161,16 @@ def test_gather_bwd_rejects_before_launch():
 
 
 def test_gather_bwd_workspace_size():
-    # two (key, position) arrays of 4-byte words for the radix passes and two
-    # fp64 partial rows per chunk of 64 sorted entries, plus the (smaller)
-    # digit histograms
-    n = eng.engram_gather_bwd_workspace_size(65536, 2, 8, 64)
+    # two (key, position) arrays of 4-byte words for the list and its radix
+    # passes, two fp64 partial rows per chunk of 64 list entries and two bits
+    # per table row, plus the (smaller) histograms and counts
+    R = 16_000_000
+    n = eng.engram_gather_bwd_workspace_size(65536, 2, 8, 64, R)
     N = 65536 * 16
-    core = 16 * N + 2 * (N // 64) * 64 * 8
+    core = 16 * N + 2 * (N // 64) * 64 * 8 + 2 * R // 8
     assert core <= n <= 2 * core
-    assert eng.engram_gather_bwd_workspace_size(0, 2, 8, 64) == 0
+    assert eng.engram_gather_bwd_workspace_size(0, 2, 8, 64, R) == 0
     with pytest.raises(eng.EngramError):
-        eng.engram_gather_bwd_workspace_size(4, 2, 8, 12)
+        eng.engram_gather_bwd_workspace_size(4, 2, 8, 12, R)
+    with pytest.raises(eng.EngramError):
+        eng.engram_gather_bwd_workspace_size(4, 2, 8, 64, 2**32)
