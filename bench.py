@@ -37,11 +37,16 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Engram gate fwd+bwd tokens/s and HBM GB/s (% of B200 peak) at H=7168"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["engram_conditional_memory_hash_b200/csrc/gate_kernels.cuh",
-                  "engram_conditional_memory_hash_b200/csrc/hash_gather.cuh",
-                  "engram_conditional_memory_hash_b200/csrc/gather_bwd.cuh",
-                  "engram_conditional_memory_hash_b200/csrc/common.cuh",
-                  "engram_conditional_memory_hash_b200/csrc/engram_abi.cu"]
+_CSRC = "engram_conditional_memory_hash_b200/csrc/"
+# the sources that define each kernel and its launch (a change to any of them
+# makes the committed DRAM counters of that kernel stale)
+KERNEL_SOURCES = {
+    "hash_gather": ["hash_gather.cuh", "common.cuh", "engram_abi.cu"],
+    "gate_fwd": ["gate_kernels.cuh", "common.cuh", "engram_abi.cu"],
+    "gate_bwd": ["gate_kernels.cuh", "common.cuh", "engram_abi.cu"],
+    "grad_w_reduce": ["gate_kernels.cuh", "common.cuh", "engram_abi.cu"],
+    "gather_bwd": ["gather_bwd.cuh", "gather_bwd_abi.inl", "hash_gather.cuh", "common.cuh"],
+}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -63,10 +68,10 @@ def algorithmic_bytes(T: int, H: int, L: int, J: int, D: int, G: int) -> dict:
     }
 
 
-def source_digest() -> str:
+def source_digest(kernel: str) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
+    for rel in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, _CSRC + rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
@@ -90,7 +95,7 @@ def committed_traffic(kernel: str, units_per_launch: int):
     except Exception:
         return None
     e = d.get(kernel)
-    if not e or e.get("source_digest") != source_digest():
+    if not e or e.get("source_digest") != source_digest(kernel):
         return None
     per_unit = e["dram_bytes"] / e["units"]
     return per_unit * units_per_launch
@@ -381,8 +386,9 @@ def run_ours(args):
         gb_bytes = T * L * J * (8 + 2 * D) + uniq * 2 * 4 * D
         gbs = gb_bytes / (us / 1e6) / 1e9
         gbwd = {"us": round(us, 2), "algorithmic_bytes": gb_bytes, "GB/s": round(gbs, 1),
-                "frac": round(gbs / peak, 4), "unique_rows": uniq, "entries": T * L * J,
-                "launches": 16,
+                "frac": round(gbs / peak, 4), "traffic": committed_traffic("gather_bwd", T),
+                "unique_rows": uniq, "entries": T * L * J,
+                "launches": 12,
                 "what": "engram_gather_bwd on the step's indices: rows read once updated in "
                         "place, the rest listed, radix-sorted by row and summed in fp64; fp32 "
                         "table-gradient update; median of 10 calls"}
@@ -481,8 +487,10 @@ def run_ours(args):
         n = 64
         rate, secs, cores = oracle_sample_rate(w, hin, gin, n)
         target = args.cpu_seconds
-        if secs < target:
-            n = int(min(w.T, max(n, n * target / max(secs, 1e-3))))
+        for _ in range(3):   # small samples overstate the per-token cost: refine the size
+            if secs >= 0.8 * target or n >= w.T:
+                break
+            n = int(min(w.T, max(n, n * 1.1 * target / max(secs, 1e-3))))
             rate, secs, cores = oracle_sample_rate(w, hin, gin, n)
         cpu = {"value": round(rate, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"first {n} tokens of the workload (hash+gather, gate fwd+bwd with "
@@ -529,6 +537,50 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+# ------------------------------------------- gather backward on its own --
+
+def run_gather_bwd_only(args):
+    """Profiling aid: engram_gather_bwd alone on the workload's hash indices
+    (no gate tensors, no table values on the device), optionally over tables
+    from another prime base (--prime-base) so that a full ncu capture holds a
+    few GB.  Prints one JSON line describing this auxiliary measurement."""
+    import torch
+
+    import engram_conditional_memory_hash_b200 as eng
+    from engram_conditional_memory_hash_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workload(args)
+    if args.prime_base:
+        w = dataclasses.replace(w, prime_base=args.prime_base)
+    T, L, J, D = w.T, w.L, w.J, w.D
+    h = inputs.hash_inputs(w, with_tables=False)
+    idx, _ = eng.engram_hash_gather(torch.from_numpy(h["tokens"]).to(dev), h["multipliers"],
+                                    h["ngram_n"], h["table_sizes"], None, pad_id=h["pad_id"],
+                                    want_rows=False)
+    d_rows = torch.from_numpy(inputs.gather_grad_inputs(w).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    R = int(h["table_sizes"].sum())
+    d_tables = torch.zeros((R, D), dtype=torch.float32, device=dev)
+    ws = torch.empty((eng.engram_gather_bwd_workspace_size(T, L, J, D, R),), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ts = []
+    for it in range(args.warmup + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        eng.engram_gather_bwd(idx, h["table_sizes"], d_rows, d_tables, workspace=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if it >= args.warmup:
+            ts.append(e0.elapsed_time(e1))
+    assert eng.engram_read_device_error() == 0
+    us = float(np.median(ts)) * 1e3
+    print(json.dumps({"part": "gather_bwd", "workload": w.name, "T": T, "rows": R, "D": D,
+                      "us": round(us, 2), "calls": args.steps, "warmup": args.warmup}), flush=True)
 
 
 # ----------------------------------------------------------- reference arm --
@@ -590,9 +642,15 @@ def main():
     ap.add_argument("--no-gather-bwd", dest="gather_bwd", action="store_false",
                     help="skip the separate engram_gather_bwd measurement")
     ap.add_argument("--ref-tokens", type=int, default=32)
+    ap.add_argument("--part", choices=["all", "gather_bwd"], default="all",
+                    help="gather_bwd: time engram_gather_bwd alone (profiling aid)")
+    ap.add_argument("--prime-base", type=int, default=0,
+                    help="with --part gather_bwd: tables of the primes from this base")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.impl == "reference":
+    if args.part == "gather_bwd":
+        run_gather_bwd_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
