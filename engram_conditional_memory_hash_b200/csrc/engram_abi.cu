@@ -422,11 +422,11 @@ engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t G, int32_t 
     if (!aligned(w_partial, 4) || !aligned(dwh, 4) || !aligned(dwe, 4) || !aligned(wh, 2) || !aligned(we, 2))
         return fail(ENGRAM_ERR_INVALID_ARG, "misaligned pointer");
     const unsigned blocks = (unsigned)((H + 31) / 32);
-    engram::grad_w_reduce_kernel<<<blocks, engram::kReduceThreads, 0,
-                                   reinterpret_cast<cudaStream_t>(stream)>>>(
-        w_partial, G, H, static_cast<const __nv_bfloat16 *>(wh), static_cast<const __nv_bfloat16 *>(we),
-        dwh, dwe);
-    cudaError_t e = cudaGetLastError();
+    // programmatic launch: scheduled while the backward kernel drains
+    const cudaError_t e = launch_pdl(engram::grad_w_reduce_kernel, blocks, (unsigned)engram::kReduceThreads,
+                                     reinterpret_cast<cudaStream_t>(stream), w_partial, G, H,
+                                     static_cast<const __nv_bfloat16 *>(wh),
+                                     static_cast<const __nv_bfloat16 *>(we), dwh, dwe);
     if (e != cudaSuccess) return cuda_fail(e, "grad_w_reduce launch");
     return ENGRAM_OK;
 }

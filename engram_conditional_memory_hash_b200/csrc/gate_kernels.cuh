@@ -432,6 +432,10 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
         }
     }
 
+    // The weight-gradient reduction launched after this kernel may now be
+    // scheduled (it waits for this whole grid before it reads the partials).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
     // Level one of the weight-gradient reduction: this CTA's partial row.
     float4 *prow = reinterpret_cast<float4 *>(w_partial + (int64_t)blockIdx.x * H);
 #pragma unroll
@@ -460,6 +464,9 @@ grad_w_reduce_kernel(const float *__restrict__ w_partial, int64_t G, int H,
 {
     __shared__ float part[kReduceWarps][33];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // launched with programmatic stream serialisation: wait for the backward
+    // kernel that wrote the partials (a no-op after any other predecessor)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int col = blockIdx.x * 32 + lane;
     float a = 0.f;
     if (col < H) {
