@@ -10,11 +10,13 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "engram.h"
 
 #include "common.cuh"
+#include "gate_generic.cuh"
 #include "gate_kernels.cuh"
 #include "gather_bwd.cuh"
 #include "hash_gather.cuh"
@@ -185,12 +187,40 @@ engram_status_t check_gate_common(int64_t T, int32_t H, float eps, float scalar)
 {
     if (T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
     if (T > (int64_t(1) << 40)) return fail(ENGRAM_ERR_UNSUPPORTED, "T=%lld too large", (long long)T);
-    if (H < 8 || H % 8 != 0 || H > kGateMaxH)
-        return fail(ENGRAM_ERR_UNSUPPORTED, "H=%d: must be a multiple of 8 in [8, %d]", H, kGateMaxH);
+    if (H < 1 || H > engram::kGenMaxH)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "H=%d not in [1, %d]", H, engram::kGenMaxH);
     if (!std::isfinite(eps) || eps < 0.f) return fail(ENGRAM_ERR_INVALID_ARG, "eps must be finite and >= 0");
     if (!std::isfinite(scalar)) return fail(ENGRAM_ERR_INVALID_ARG, "scalar must be finite");
     return ENGRAM_OK;
 }
+
+// The tuned gate kernels stream whole rows with 16-byte bulk copies: H a
+// multiple of 8 up to kGateMaxH and every bf16 tensor on a 16-byte boundary.
+// Any other H (up to kGenMaxH) or 2-byte alignment goes to gate_generic.cuh.
+bool gate_tuned(int H, std::initializer_list<const void *> ptrs)
+{
+    if (H % 8 != 0 || H > kGateMaxH) return false;
+    for (const void *p : ptrs)
+        if (p != nullptr && !aligned(p, 16)) return false;
+    return true;
+}
+
+// The generic kernels read rows with 16-byte vectors when every token tensor
+// starts at the same offset from a 16-byte boundary.
+bool same_phase(std::initializer_list<const void *> ptrs)
+{
+    int phase = -1;
+    for (const void *p : ptrs) {
+        if (p == nullptr) continue;
+        const int ph = (int)(reinterpret_cast<uintptr_t>(p) & 15u);
+        if (phase < 0) phase = ph;
+        else if (ph != phase) return false;
+    }
+    return true;
+}
+
+// CTAs of the generic gate kernels: up to 8 per SM, never more than tokens.
+int64_t generic_grid(const DeviceInfo &d, int64_t T) { return std::max<int64_t>(1, std::min<int64_t>(T, (int64_t)d.sms * 8)); }
 
 // -------------------------------------------------------------- launches ----
 
@@ -330,13 +360,25 @@ engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, con
     if (T == 0) return ENGRAM_OK;
     if (!x || !k || !v || !wh || !we || !out)
         return fail(ENGRAM_ERR_INVALID_ARG, "x, k, v, wh, we and out are required");
-    if (!aligned(x, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(wh, 16) || !aligned(we, 16) ||
-        !aligned(out, 16))
-        return fail(ENGRAM_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+    if (!aligned(x, 2) || !aligned(k, 2) || !aligned(v, 2) || !aligned(wh, 2) || !aligned(we, 2) ||
+        !aligned(out, 2))
+        return fail(ENGRAM_ERR_INVALID_ARG, "bf16 tensors must be 2-byte aligned");
     if (gate && !aligned(gate, 4)) return fail(ENGRAM_ERR_INVALID_ARG, "gate must be 4-byte aligned");
 
     DeviceInfo dev;
     if ((st = device_info(&dev)) != ENGRAM_OK) return st;
+    if (!gate_tuned(H, {x, k, v, wh, we, out})) {
+        auto kern = same_phase({x, k, v, out}) ? engram::gate_generic_fwd_kernel<true>
+                                               : engram::gate_generic_fwd_kernel<false>;
+        kern<<<(unsigned)generic_grid(dev, T), engram::kGenThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+            static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(k),
+            static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(wh),
+            static_cast<const __nv_bfloat16 *>(we), T, H, eps, scalar, static_cast<__nv_bfloat16 *>(out),
+            gate);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "gate_fwd launch");
+        return ENGRAM_OK;
+    }
     GateLaunch g;
     if ((st = gate_fwd_plan(dev, H, &g)) != ENGRAM_OK) return st;
     const int64_t grid = std::min<int64_t>(T, (int64_t)dev.sms * g.ctas_per_sm);
@@ -359,12 +401,13 @@ engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, con
 
 int64_t engram_gate_bwd_num_partials(int64_t T, int32_t H)
 {
-    if (H < 8 || H % 8 != 0 || H > kGateMaxH) {
-        fail(ENGRAM_ERR_UNSUPPORTED, "H=%d: must be a multiple of 8 in [8, %d]", H, kGateMaxH);
+    if (H < 1 || H > engram::kGenMaxH) {
+        fail(ENGRAM_ERR_UNSUPPORTED, "H=%d not in [1, %d]", H, engram::kGenMaxH);
         return -1;
     }
     DeviceInfo dev;
     if (device_info(&dev) != ENGRAM_OK) return -1;
+    if (!gate_tuned(H, {})) return generic_grid(dev, T);
     GateLaunch g;
     if (gate_bwd_plan(dev, H, &g) != ENGRAM_OK) return -1;
     const int64_t full = (int64_t)dev.sms * g.ctas_per_sm;
@@ -385,16 +428,33 @@ engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void 
     if (T > 0 && (!grad_out || !x || !k || !v || !dx || !dk || !dv))
         return fail(ENGRAM_ERR_INVALID_ARG, "every tensor argument of engram_gate_bwd is required");
     if (G < 1 || G > 0x7fffffff) return fail(ENGRAM_ERR_INVALID_ARG, "G=%lld not in [1, 2^31-1]", (long long)G);
-    if (!aligned(grad_out, 16) || !aligned(x, 16) || !aligned(k, 16) || !aligned(v, 16) ||
-        !aligned(wh, 16) || !aligned(we, 16) || !aligned(dx, 16) || !aligned(dk, 16) ||
-        !aligned(dv, 16) || !aligned(w_partial, 16))
-        return fail(ENGRAM_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    if (!aligned(grad_out, 2) || !aligned(x, 2) || !aligned(k, 2) || !aligned(v, 2) || !aligned(wh, 2) ||
+        !aligned(we, 2) || !aligned(dx, 2) || !aligned(dk, 2) || !aligned(dv, 2))
+        return fail(ENGRAM_ERR_INVALID_ARG, "bf16 tensors must be 2-byte aligned");
+    if (!aligned(w_partial, 4)) return fail(ENGRAM_ERR_INVALID_ARG, "w_partial must be 4-byte aligned");
 
     DeviceInfo dev;
     if ((st = device_info(&dev)) != ENGRAM_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!gate_tuned(H, {grad_out, x, k, v, wh, we, dx, dk, dv, w_partial})) {
+        auto kern = same_phase({grad_out, x, k, v, dx, dk, dv}) ? engram::gate_generic_bwd_kernel<true>
+                                                                 : engram::gate_generic_bwd_kernel<false>;
+        const size_t smem = H <= engram::kGenSmemPartial ? (size_t)H * 4 : 0;
+        cudaError_t e0 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              (int)(engram::kGenSmemPartial * 4));
+        if (e0 != cudaSuccess) return cuda_fail(e0, "cudaFuncSetAttribute");
+        kern<<<(unsigned)G, engram::kGenThreads, smem, s>>>(
+            static_cast<const __nv_bfloat16 *>(grad_out), static_cast<const __nv_bfloat16 *>(x),
+            static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v),
+            static_cast<const __nv_bfloat16 *>(wh), static_cast<const __nv_bfloat16 *>(we), T, H, eps, scalar,
+            static_cast<__nv_bfloat16 *>(dx), static_cast<__nv_bfloat16 *>(dk),
+            static_cast<__nv_bfloat16 *>(dv), w_partial);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "gate_bwd launch");
+        return ENGRAM_OK;
+    }
     GateLaunch g;
     if ((st = gate_bwd_plan(dev, H, &g)) != ENGRAM_OK) return st;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     auto args = [&](auto kern) -> engram_status_t {
         kern<<<(unsigned)G, g.threads, g.smem, s>>>(
             static_cast<const uint4 *>(grad_out), static_cast<const uint4 *>(x),

@@ -19,9 +19,14 @@
  *   - Every compute call is asynchronous on `stream` (NULL: the legacy default
  *     stream) and never synchronises.  Outputs are valid once the stream has
  *     reached the call.
- *   - "bf16" tensors are contiguous, row-major arrays of IEEE bfloat16.  Every
- *     bf16 tensor must start on a 16-byte boundary; H must be a multiple of 8
- *     (one 16-byte vector holds 8 bf16 values).
+ *   - "bf16" tensors are contiguous, row-major arrays of IEEE bfloat16.  The
+ *     gate calls take any hidden size H in [1, 65536] and bf16 tensors on any
+ *     2-byte boundary: when H is a multiple of 8 up to 8192 and every bf16
+ *     tensor (and the fp32 partial rows) starts on a 16-byte boundary, the
+ *     kernels tuned for the pages' sizes run (whole rows moved with 16-byte
+ *     bulk copies); otherwise generic kernels compute the same formulas with
+ *     plain loads, two passes over each token's rows.  The hash/gather calls
+ *     keep their own alignment rules, stated below.
  *   - Errors: arguments are checked before anything is launched; a failing
  *     check returns ENGRAM_ERR_INVALID_ARG (bad pointer, size or alignment) or
  *     ENGRAM_ERR_UNSUPPORTED (a size this build does not handle) and launches
@@ -170,12 +175,12 @@ ENGRAM_API engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int3
  *     gate = sigmoid(sign(s) sqrt(|s|)),   out = x + gate * v
  * Accumulation is fp32; out is rounded to bf16 (nearest even).
  *
- * x, k, v     device, bf16 [T*H], row-major [T][H], 16-byte aligned.
- * wh, we      device, bf16 [H], 16-byte aligned.
+ * x, k, v     device, bf16 [T*H], row-major [T][H], 2-byte aligned.
+ * wh, we      device, bf16 [H], 2-byte aligned.
  * T           >= 0 tokens (0 launches nothing; the pointers may then be NULL).
- * H           hidden size: multiple of 8, 8..8192.
+ * H           hidden size, 1..65536 (see the conventions for which kernels run).
  * eps         >= 0, finite.   scalar  finite (normally 1/sqrt(H)).
- * out         device, bf16 [T*H], 16-byte aligned (may not alias the inputs).
+ * out         device, bf16 [T*H], 2-byte aligned (may not alias the inputs).
  * gate        device, fp32 [T], 4-byte aligned, or NULL to skip it.
  */
 ENGRAM_API engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, const void *wh,
@@ -204,11 +209,11 @@ ENGRAM_API int64_t engram_gate_bwd_num_partials(int64_t T, int32_t H);
  * CTA p of G handles tokens p, p+G, p+2G, ... in that order, so the partials
  * (and everything else) are bitwise reproducible for a given G.
  *
- * grad_out, x, k, v  device, bf16 [T*H], 16-byte aligned.
- * wh, we             device, bf16 [H], 16-byte aligned.
+ * grad_out, x, k, v  device, bf16 [T*H], 2-byte aligned.
+ * wh, we             device, bf16 [H], 2-byte aligned.
  * T >= 0, H as in engram_gate_fwd, eps/scalar as passed to the forward.
- * dx, dk, dv         device, bf16 [T*H], 16-byte aligned (no aliasing).
- * w_partial          device, fp32 [G*H], 16-byte aligned; fully overwritten
+ * dx, dk, dv         device, bf16 [T*H], 2-byte aligned (no aliasing).
+ * w_partial          device, fp32 [G*H], 4-byte aligned; fully overwritten
  *                    (rows of CTAs without tokens are written as zeros, so
  *                    T == 0 yields all-zero partials; the token tensors may
  *                    then be NULL).

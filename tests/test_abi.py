@@ -49,14 +49,13 @@ def _fwd(L, T=4, H=64, ptr=16, out=16, eps=1e-6, scalar=0.125):
 
 def test_gate_fwd_rejects_before_launch():
     L = eng.lib()
-    assert _fwd(L, H=12) == UNSUPPORTED           # not a multiple of 8
     assert _fwd(L, H=0) == UNSUPPORTED
-    assert _fwd(L, H=8200) == UNSUPPORTED         # beyond the supported range
-    assert b"multiple of 8" in L.engram_last_error()
+    assert _fwd(L, H=65544) == UNSUPPORTED        # beyond the supported range
+    assert b"not in [1, 65536]" in L.engram_last_error()
     assert _fwd(L, T=-1) == INVALID
     assert _fwd(L, ptr=None) == INVALID
     assert _fwd(L, out=None) == INVALID
-    assert _fwd(L, ptr=24) == INVALID               # not 16-byte aligned
+    assert _fwd(L, ptr=25) == INVALID               # bf16 at an odd address
     assert b"aligned" in L.engram_last_error()
     assert _fwd(L, eps=float("nan")) == INVALID
     assert _fwd(L, eps=-1.0) == INVALID
@@ -73,9 +72,10 @@ def test_gate_bwd_rejects_before_launch():
 
     assert bwd(G=0) == INVALID
     assert bwd(G=2**31) == INVALID
-    assert bwd(H=20) == UNSUPPORTED
+    assert bwd(H=0) == UNSUPPORTED and bwd(H=70000) == UNSUPPORTED
     assert bwd(ptr=None) == INVALID
-    assert bwd(part=ctypes.c_void_p(20)) == INVALID
+    assert bwd(ptr=ctypes.c_void_p(17)) == INVALID                  # bf16 at an odd address
+    assert bwd(part=ctypes.c_void_p(18)) == INVALID                 # fp32 partials not 4-aligned
 
 
 def test_grad_w_reduce_rejects_before_launch():

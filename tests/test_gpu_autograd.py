@@ -67,3 +67,35 @@ def test_module_trains_a_step():
     before = layer.wh.detach().clone()
     opt.step()
     assert not torch.equal(before, layer.wh.detach())
+
+
+def test_hash_gather_function_and_module(oracle_lib):
+    # the tiny workload through EngramMemory: rows equal the direct call
+    # (bit-exact), the tables' gradient equals engram_gather_bwd's fp32 result
+    # rounded to bf16, and that agrees with the oracle's gather backward
+    from engram_conditional_memory_hash_b200.autograd import EngramMemory
+    w = inputs.WORKLOADS["tiny"]
+    h = inputs.hash_inputs(w)
+    mem = EngramMemory(h["table_sizes"], w.D, h["ngram_n"], h["multipliers"], pad_id=h["pad_id"],
+                       device="cuda")
+    with torch.no_grad():
+        mem.tables.copy_(to_dev_bf16(h["tables"]).view(-1, w.D))
+    tokens = torch.from_numpy(h["tokens"]).cuda()
+    rows = mem(tokens)
+    d_rows = to_dev_bf16(inputs.gather_grad_inputs(w)).view(rows.shape)
+    rows.backward(d_rows)
+    torch.cuda.synchronize()
+
+    idx, want_rows = eng.engram_hash_gather(tokens, h["multipliers"], h["ngram_n"],
+                                            h["table_sizes"], mem.tables.detach(),
+                                            pad_id=h["pad_id"])
+    assert torch.equal(rows.detach().view(torch.int16), want_rows.view(torch.int16))
+    d_tab = eng.engram_gather_bwd(idx, h["table_sizes"], d_rows)
+    torch.cuda.synchronize()
+    assert mem.tables.grad.dtype == torch.bfloat16
+    assert torch.equal(mem.tables.grad.view(torch.int16), d_tab.to(torch.bfloat16).view(torch.int16))
+    ref = oracle_lib.engram_gather_bwd(idx.cpu().numpy(), h["table_sizes"],
+                                       inputs.gather_grad_inputs(w))
+    got = mem.tables.grad.float().cpu().double().numpy()
+    # bf16 rounding of an exactly summed fp32 value: within 2^-8 relative
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)

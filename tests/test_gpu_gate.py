@@ -114,17 +114,40 @@ def test_deterministic(oracle_lib):
         assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
 
 
-def test_misaligned_and_bad_shapes_rejected():
-    H = 64
-    x = torch.zeros(5 * H + 8, dtype=torch.bfloat16, device="cuda")
-    xs = x[4:4 + 4 * H].view(4, H)   # 8-byte offset
-    w1 = torch.ones(H, dtype=torch.bfloat16, device="cuda")
+@pytest.mark.parametrize("T,H", [(3, 1), (5, 7), (129, 100), (40, 1001), (17, 8200), (9, 16384),
+                                 (3, 65536)])
+def test_generic_hidden_sizes(oracle_lib, T, H):
+    # H not a multiple of 8 or above 8192: the generic kernels; every output
+    # against the oracle, and G covering more and fewer CTAs than tokens
+    w = inputs.Workload("generic", 180 + H % 23, B=1, S=T, H=H, backward=True)
+    gi = inputs.gate_inputs(w)
+    _check_all(oracle_lib, gi, _gpu_path(_dev(gi)))
+    _check_all(oracle_lib, gi, _gpu_path(_dev(gi), G=max(1, T // 2)))
+    assert eng.engram_read_device_error() == 0
+
+
+def test_unaligned_tensors_take_the_generic_path(oracle_lib):
+    # bf16 tensors starting 2 and 8 bytes past a 16-byte boundary (H = 64):
+    # the tuned kernels need 16-byte aligned rows, the generic ones do not
+    T, H = 37, 64
+    w = inputs.Workload("unaligned", 210, B=1, S=T, H=H, backward=True)
+    gi = inputs.gate_inputs(w)
+    for off in (1, 4):
+        t = {}
+        for n, a in gi.items():
+            flat = to_dev_bf16(a).reshape(-1)
+            buf = torch.zeros(flat.numel() + 8, dtype=torch.bfloat16, device="cuda")
+            buf[off:off + flat.numel()] = flat
+            t[n] = buf[off:off + flat.numel()].view(a.shape)
+        assert t["x"].data_ptr() % 16 != 0
+        _check_all(oracle_lib, gi, _gpu_path(t))
+
+
+def test_bad_shapes_rejected():
+    big = torch.zeros(2, 65544, dtype=torch.bfloat16, device="cuda")
+    w1 = torch.ones(65544, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(eng.EngramError):
-        eng.engram_gate_fwd(xs, xs, xs, w1, w1)
-    bad = torch.zeros(4, 12, dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(eng.EngramError):
-        eng.engram_gate_fwd(bad, bad, bad, torch.ones(12, dtype=torch.bfloat16, device="cuda"),
-                            torch.ones(12, dtype=torch.bfloat16, device="cuda"))
+        eng.engram_gate_fwd(big, big, big, w1, w1)
 
 
 def test_empty_tokens():
