@@ -158,6 +158,35 @@ def test_empty_and_argument_errors():
         eng.engram_gather_bwd(idx, sizes, d_rows, d_tables, workspace=small)
 
 
+def test_four_radix_passes(oracle_lib):
+    # 16 tables of ~4.19M rows (67M rows in all, more than 2^24): row keys need
+    # four 8-bit radix passes; a Zipf-like skew makes many rows repeat.  D = 8
+    # keeps the fp32 table gradient at 2.1 GB.  Checked on row windows around
+    # the hottest rows and at random, plus the touched-row property.
+    r = np.random.default_rng(44)
+    L, J, T, D = 2, 8, 4096, 8
+    sizes = inputs.consecutive_primes(4194301, L * J).reshape(L, J)
+    R = int(sizes.sum())
+    assert R > 2 ** 24 * 3
+    idx_np = np.minimum((r.pareto(0.8, size=(T, L, J)) * 50).astype(np.int64), sizes[None] - 1)
+    d_rows = inputs.f32_to_bf16_bits(r.standard_normal((T, L, J, D)).astype(np.float32))
+    d_tables = torch.zeros((R, D), dtype=torch.float32, device="cuda")
+    eng.engram_gather_bwd(torch.from_numpy(idx_np).cuda(), sizes, to_dev_bf16(d_rows), d_tables)
+    assert eng.engram_read_device_error() == 0
+    first = np.concatenate([[0], np.cumsum(sizes.ravel())[:-1]])
+    rows = (idx_np.reshape(-1, L * J) + first[None]).ravel()
+    uniq, counts = np.unique(rows, return_counts=True)
+    assert counts.max() > 50
+    hot = uniq[np.argsort(counts)[-3:]]
+    for lo in [0, R - 64] + [int(x) - 2 for x in hot] + [int(x) for x in r.integers(0, R - 64, 3)]:
+        lo = max(0, lo)
+        hi = min(R, lo + 64)
+        want, tol, touched = _expect(oracle_lib, idx_np, sizes, d_rows, np.zeros((hi - lo, D)), lo, hi)
+        _check(d_tables[lo:hi], want, tol, touched, np.zeros((hi - lo, D)))
+    nonzero = (d_tables != 0).any(dim=1).nonzero().flatten().cpu().numpy()
+    np.testing.assert_array_equal(nonzero, uniq)
+
+
 def test_full_path_size_sampled(oracle_lib):
     # the full-path workload as the benchmark runs it: 65536 Zipf tokens, 16
     # tables of ~1M rows x 64; d_tables (4.1 GB fp32) checked on windows of rows
