@@ -119,25 +119,13 @@ __device__ __forceinline__ void gate_pipeline_start(unsigned char *smem, uint32_
     }
 }
 
-#ifndef ENGRAM_COMBINE_SHUFFLE
-#define ENGRAM_COMBINE_SHUFFLE 0
-#endif
-
-// Sum of the per-warp partials of one token, in a fixed order: every thread
-// either adds the nwarps entries in warp order, or (ENGRAM_COMBINE_SHUFFLE)
-// lane q takes warp q's entry and a shuffle tree adds them.
+// Sum of the per-warp partials of one token, in warp order (a fixed order):
+// every thread adds the nwarps entries itself, which keeps the per-token
+// critical path short (a shuffle tree over the warps' entries was measured
+// slower: it lengthens the chain every token waits on).
 __device__ __forceinline__ void combine_partials(const float4 *rb, const double *rbd, int nwarps,
-                                                 int lane, float4 &r, double &A)
+                                                 float4 &r, double &A)
 {
-#if ENGRAM_COMBINE_SHUFFLE
-    r = lane < nwarps ? rb[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-    A = lane < nwarps ? rbd[lane] : 0.0;
-    r.x = warp_sum(r.x);
-    r.y = warp_sum(r.y);
-    r.z = warp_sum(r.z);
-    A = warp_sum_f64(A);
-#else
-    (void)lane;
     r = make_float4(0.f, 0.f, 0.f, 0.f);
     A = 0.0;
     for (int q = 0; q < nwarps; ++q) {
@@ -147,7 +135,6 @@ __device__ __forceinline__ void combine_partials(const float4 *rb, const double 
         r.z += t.z;
         A += rbd[q];
     }
-#endif
 }
 
 // Per-token gate from the reduced statistics.
@@ -269,7 +256,7 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
 
         float4 r;
         double A;
-        combine_partials(rb, rbd, nwarps, lane, r, A);
+        combine_partials(rb, rbd, nwarps, r, A);
         const GateScalars c = gate_scalars(r.x, r.y, A, inv_h, eps, scalar);
 
         const int64_t row = first + i * G;
@@ -393,7 +380,7 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
 
         float4 r;
         double A;
-        combine_partials(rb, rbd, nwarps, lane, r, A);
+        combine_partials(rb, rbd, nwarps, r, A);
         const float Sg = r.z;
         const GateScalars c = gate_scalars(r.x, r.y, A, inv_h, eps, scalar);
         // chain rule through sigmoid, signed_sqrt (|s| clamped at 1e-6), scalar
