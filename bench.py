@@ -495,10 +495,13 @@ def run_ours(args):
         cpu = {"value": round(rate, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"first {n} tokens of the workload (hash+gather, gate fwd+bwd with "
                          f"weight gradients), {secs:.1f} s of fp64 CPU work"}
-        # the same oracle on one host thread, on a sample sized for about the
-        # same CPU time
-        n1 = max(64, int(n / max(1, cores)))
+        # the same oracle on one host thread, on a sample sized for about half
+        # the all-cores run's time
+        n1 = 1024
         rate1, secs1, _ = oracle_sample_rate(w, hin, gin, n1, threads=1)
+        if secs1 < 0.4 * target and n1 < w.T:
+            n1 = int(min(w.T, n1 * 0.5 * target / max(secs1, 1e-3)))
+            rate1, secs1, _ = oracle_sample_rate(w, hin, gin, n1, threads=1)
         import oracle as _oracle
         _oracle.default().set_threads(cores)
         cpu["one_thread"] = {"value": round(rate1, 1), "unit": "tokens/s", "cores": 1,
