@@ -603,6 +603,12 @@ def run_reference(args):
     w = workload(args)
     hin, gin = host_inputs(w, 0)
     n = args.ref_tokens
+    if n <= 0:
+        # size each step's sample so that the whole run (warm-up and timed
+        # steps) takes about --ref-seconds of CPU time
+        rate, _, _ = oracle_sample_rate(w, hin, gin, 256)
+        per_step = args.ref_seconds / max(1, args.warmup + args.steps)
+        n = int(min(w.T, max(32, rate * per_step)))
     rates, secs_all = [], []
     cores = 0
     for i in range(args.warmup + args.steps):
@@ -652,7 +658,10 @@ def main():
                     help="skip the uniform-id hash_gather control measurement")
     ap.add_argument("--no-gather-bwd", dest="gather_bwd", action="store_false",
                     help="skip the separate engram_gather_bwd measurement")
-    ap.add_argument("--ref-tokens", type=int, default=32)
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="tokens per reference-arm step (0: sized from --ref-seconds)")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="CPU time the whole reference-arm run aims at")
     ap.add_argument("--part", choices=["all", "gather_bwd"], default="all",
                     help="gather_bwd: time engram_gather_bwd alone (profiling aid)")
     ap.add_argument("--prime-base", type=int, default=0,
