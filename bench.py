@@ -210,6 +210,24 @@ def workload(args):
     return w
 
 
+def time_calls(call, stream, dev, warmup: int, calls: int) -> float:
+    """Microseconds per call of `call` (which enqueues GPU work on `stream`):
+    `warmup` calls, then `calls` calls enqueued back to back between two CUDA
+    events, so that the host's time to issue a call overlaps the GPU's work
+    on the previous one."""
+    import torch
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(calls):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) * 1e3 / calls
+
+
 def host_inputs(w, rank: int):
     from engram_conditional_memory_hash_b200 import inputs
     wr = dataclasses.replace(w, index=w.index + 1000 * rank)
@@ -336,14 +354,17 @@ def run_ours(args):
         from engram_conditional_memory_hash_b200 import inputs as _inp
         utok = torch.from_numpy(_inp.uniform_ids(w.seed, 99, (w.B, w.S), 0, w.vocab)).to(dev)
         flush = torch.empty(2 * 126 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        # its own outputs: the step's indices in buf0 stay those of the step's
+        # tokens (the gather backward below runs on them)
+        uidx, urows = torch.empty_like(buf0["idx"]), torch.empty_like(buf0["rows"])
         ts = []
         for it in range(13):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             eng.engram_hash_gather(utok, hin["multipliers"], hin["ngram_n"], hin["table_sizes"],
-                                   tables, pad_id=hin["pad_id"], idx_out=buf0["idx"],
-                                   rows_out=buf0["rows"], stream=stream)
+                                   tables, pad_id=hin["pad_id"], idx_out=uidx,
+                                   rows_out=urows, stream=stream)
             e1.record(stream)
             torch.cuda.synchronize(dev)
             if it >= 3:
@@ -352,7 +373,7 @@ def run_ours(args):
         gbs = ab["hash_gather"] / (us / 1e6) / 1e9
         uniform = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
                    "ids": f"uniform over [0, {w.vocab}), L2 flushed before each launch"}
-        del flush
+        del flush, uidx, urows
 
     # Gather backward (the transpose of the gather: row gradients summed into
     # the fp32 table gradient), timed on its own: it is not one of the four
@@ -371,17 +392,9 @@ def run_ours(args):
         first = torch.from_numpy(np.concatenate(
             [[0], np.cumsum(hin["table_sizes"].ravel())[:-1]])).to(dev)
         uniq = int(torch.unique(buf0["idx"].view(T, L * J) + first[None]).numel())
-        ts = []
-        for it in range(13):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            eng.engram_gather_bwd(buf0["idx"], hin["table_sizes"], d_rows, d_tables, workspace=ws,
-                                  stream=stream)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            if it >= 3:
-                ts.append(e0.elapsed_time(e1))
-        us = float(np.median(ts)) * 1e3
+        us = time_calls(lambda: eng.engram_gather_bwd(buf0["idx"], hin["table_sizes"], d_rows,
+                                                      d_tables, workspace=ws, stream=stream),
+                        stream, dev, warmup=3, calls=20)
         # idx read + d_rows read + one read and one write of every touched fp32 table row
         gb_bytes = T * L * J * (8 + 2 * D) + uniq * 2 * 4 * D
         gbs = gb_bytes / (us / 1e6) / 1e9
@@ -391,7 +404,8 @@ def run_ours(args):
                 "launches": 12,
                 "what": "engram_gather_bwd on the step's indices: rows read once updated in "
                         "place, the rest listed, radix-sorted by row and summed in fp64; fp32 "
-                        "table-gradient update; median of 10 calls"}
+                        "table-gradient update; 20 calls back to back, CUDA events around "
+                        "them"}
         del d_rows, d_tables, ws
 
     kern = {}
@@ -579,17 +593,10 @@ def run_gather_bwd_only(args):
     ws = torch.empty((eng.engram_gather_bwd_workspace_size(T, L, J, D, R),), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream(dev)
-    ts = []
-    for it in range(args.warmup + args.steps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        eng.engram_gather_bwd(idx, h["table_sizes"], d_rows, d_tables, workspace=ws, stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        if it >= args.warmup:
-            ts.append(e0.elapsed_time(e1))
+    us = time_calls(lambda: eng.engram_gather_bwd(idx, h["table_sizes"], d_rows, d_tables,
+                                                  workspace=ws, stream=stream),
+                    stream, dev, warmup=args.warmup, calls=args.steps)
     assert eng.engram_read_device_error() == 0
-    us = float(np.median(ts)) * 1e3
     print(json.dumps({"part": "gather_bwd", "workload": w.name, "T": T, "rows": R, "D": D,
                       "us": round(us, 2), "calls": args.steps, "warmup": args.warmup}), flush=True)
 

@@ -108,8 +108,9 @@ __device__ __forceinline__ bool row_bit(const uint32_t *__restrict__ map, uint32
 // seen/dupmap bits of every entry's row (both bitmaps zeroed before the
 // launch): an entry that finds its row's `seen` bit already set sets the row's
 // `dupmap` bit.  Which entry arrives first does not matter: a row ends up in
-// dupmap exactly when two or more entries read it.  Entries of rows already in
-// dupmap (the hot rows of skewed inputs) skip the atomics.
+// dupmap exactly when two or more entries read it.  (Reading dupmap first to
+// skip the atomics of hot rows saves nothing: every entry is in flight at
+// once, so the check sees the bitmap before any atomic has landed.)
 __global__ void __launch_bounds__(kMarkThreads)
 gbwd_mark_kernel(const int64_t *__restrict__ idx, const __grid_constant__ GatherBwdParams p,
                  uint32_t *__restrict__ seen, uint32_t *__restrict__ dupmap)
@@ -127,7 +128,6 @@ gbwd_mark_kernel(const int64_t *__restrict__ idx, const __grid_constant__ Gather
         for (int x = 0; x < 4; ++x) {
             if (kk[x] >= p.R) continue;
             const uint32_t bit = 1u << (kk[x] & 31u);
-            if (__ldcg(&dupmap[kk[x] >> 5]) & bit) continue;
             if (atomicOr(&seen[kk[x] >> 5], bit) & bit) atomicOr(&dupmap[kk[x] >> 5], bit);
         }
     }
@@ -622,27 +622,49 @@ gbwd_segment_kernel(const uint32_t *__restrict__ keys, const uint32_t *__restric
                 }
             }
             // rows read several times.  A short run (up to kLongRun entries)
-            // is summed by its own group, its gradients loaded four at a time;
+            // is summed by its own group: the first four gradients of each of
+            // the group's U runs are requested together, the rest four at a
+            // time;
             // a long run (a hot row) by the whole warp: group g takes the
             // entries b + g, b + g + GPW, ... (four at a time) and the groups'
             // partials are combined by a butterfly over the groups (a fixed
             // order; every group ends with the same bits).  All sums are fp64;
             // the first gradient row and the table row are reloaded, from cache.
-#pragma unroll 1
-            for (int u = 0; u < U; ++u) {
-                if (!multi[u] || se[u] - sb[u] > kLongRun) continue;
-                double a[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-                for (int e = sb[u]; e < se[u]; e += 4) {
-                    uint4 q[4];
+            {
+                double a[U][8];
+                uint4 q[U][4];
+                bool sh[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    sh[u] = multi[u] && se[u] - sb[u] <= kLongRun;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) a[u][k] = 0.0;
 #pragma unroll
                     for (int x = 0; x < 4; ++x)
-                        q[x] = e + x < se[u] ? __ldg(d_rows + (int64_t)s_pos[warp][e + x] * nv + cv)
-                                             : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) add_bf16x8(a, q[x]);
+                        q[u][x] = sh[u] && sb[u] + x < se[u]
+                                      ? __ldg(d_rows + (int64_t)s_pos[warp][sb[u] + x] * nv + cv)
+                                      : make_uint4(0u, 0u, 0u, 0u);
                 }
-                finish_segment(a, comp[u], contb[u], key[u], c, cv, nv, p.D, d_tables, carry_a, carry_b,
-                               carry_list, carry_count);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) add_bf16x8(a[u], q[u][x]);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (!sh[u]) continue;
+                    for (int e = sb[u] + 4; e < se[u]; e += 4) {
+                        uint4 r4[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x)
+                            r4[x] = e + x < se[u] ? __ldg(d_rows + (int64_t)s_pos[warp][e + x] * nv + cv)
+                                                  : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) add_bf16x8(a[u], r4[x]);
+                    }
+                    finish_segment(a[u], comp[u], contb[u], key[u], c, cv, nv, p.D, d_tables, carry_a, carry_b,
+                                   carry_list, carry_count);
+                }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
