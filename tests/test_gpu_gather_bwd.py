@@ -103,6 +103,40 @@ def test_one_hot_row_per_table(oracle_lib, T):
     _check(got, want, tol, touched, init)
 
 
+def test_most_tables(oracle_lib):
+    # the largest table count the library takes (4 layers x 16 tables), every
+    # table a different size, so each entry's table offset and bound come from
+    # its own slot of the per-table parameters
+    r = np.random.default_rng(64)
+    L, J, T, D = 4, 16, 389, 32
+    sizes = inputs.consecutive_primes(211, L * J).reshape(L, J)
+    idx_np = (r.random((T, L, J)) ** 2 * sizes[None]).astype(np.int64)
+    d_rows = inputs.f32_to_bf16_bits(r.standard_normal((T, L, J, D)).astype(np.float32))
+    R = int(sizes.sum())
+    init = r.standard_normal((R, D)).astype(np.float32).astype(np.float64)
+    got = _run(torch.from_numpy(idx_np).cuda(), sizes, d_rows, init)
+    want, tol, touched = _expect(oracle_lib, idx_np, sizes, d_rows, init)
+    _check(got, want, tol, touched, init)
+
+
+def test_no_repeated_rows(oracle_lib):
+    # every entry reads its own row: all of them take the in-place update and
+    # the list of repeated rows' entries is empty (its kernels see M = 0)
+    L, J, T, D = 2, 8, 1500, 64
+    sizes = np.full((L, J), 4 * T + 1, dtype=np.int64)
+    t = np.arange(T, dtype=np.int64)[:, None, None]
+    q = np.arange(L * J, dtype=np.int64).reshape(1, L, J)
+    idx_np = (3 * t + q) % sizes[None]          # distinct within each table
+    r = np.random.default_rng(15)
+    d_rows = inputs.f32_to_bf16_bits(r.standard_normal((T, L, J, D)).astype(np.float32))
+    R = int(sizes.sum())
+    init = r.standard_normal((R, D)).astype(np.float32).astype(np.float64)
+    got = _run(torch.from_numpy(idx_np).cuda(), sizes, d_rows, init)
+    want, tol, touched = _expect(oracle_lib, idx_np, sizes, d_rows, init)
+    assert int(touched.sum()) == T * L * J
+    _check(got, want, tol, touched, init)
+
+
 def test_deterministic_and_accumulating(oracle_lib):
     w = inputs.WORKLOADS["tiny"]
     r = np.random.default_rng(3)
