@@ -171,6 +171,10 @@ engram_status_t gate_fwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
                      engram::gate_fwd_kernel<2>, engram::gate_fwd_kernel<4>, g);
 }
 
+// Thread bound of the two-vector backward variant with the larger register
+// budget (used whenever the row needs no more threads).
+constexpr int kBwdNarrowThreads = 448;
+
 // Backward: ENGRAM_BWD_VEC vectors per thread (one for rows of at most 64
 // vectors, four where two would need more than 512 threads).
 engram_status_t gate_bwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
@@ -179,6 +183,9 @@ engram_status_t gate_bwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
     int maxv = ENGRAM_BWD_VEC;
     if (nvec <= 64) maxv = 1;
     while ((nvec + maxv - 1) / maxv > engram::gate_max_threads(maxv) && maxv < 4) maxv *= 2;
+    if (maxv == 2 && (nvec + 1) / 2 <= kBwdNarrowThreads)
+        return gate_plan(d, H, 4, maxv, ENGRAM_BWD_MAX_CTAS, engram::gate_bwd_kernel<1>,
+                         engram::gate_bwd_kernel<2, kBwdNarrowThreads>, engram::gate_bwd_kernel<4>, g);
     return gate_plan(d, H, 4, maxv, ENGRAM_BWD_MAX_CTAS, engram::gate_bwd_kernel<1>,
                      engram::gate_bwd_kernel<2>, engram::gate_bwd_kernel<4>, g);
 }
@@ -465,6 +472,7 @@ engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void 
         if (e != cudaSuccess) return cuda_fail(e, "gate_bwd launch");
         return ENGRAM_OK;
     };
+    if (g.maxv == 2 && g.threads <= kBwdNarrowThreads) return args(engram::gate_bwd_kernel<2, kBwdNarrowThreads>);
     return g.maxv == 1 ? args(engram::gate_bwd_kernel<1>)
          : g.maxv == 2 ? args(engram::gate_bwd_kernel<2>)
                        : args(engram::gate_bwd_kernel<4>);

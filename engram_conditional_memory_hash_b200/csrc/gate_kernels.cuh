@@ -280,8 +280,13 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
 
 // -------------------------------------------------------------- backward ----
 
-template <int MAXV>
-__global__ void __launch_bounds__(gate_max_threads(MAXV), 1)
+// Backward kernel with MAXV vectors per thread and at most MAXT threads per
+// CTA.  The launch bound sets the register budget: at MAXV = 2 a CTA of up to
+// 448 threads (rows of up to 7168 values) may hold 144 registers per thread,
+// room for the fused weight in fp64 as well as fp32 (pass 1 then converts
+// only x·k to fp64, not w); the 512-thread variant covers rows up to 8192.
+template <int MAXV, int MAXT = gate_max_threads(MAXV)>
+__global__ void __launch_bounds__(MAXT, 1)
 gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
                 const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                 const uint4 *__restrict__ wh, const uint4 *__restrict__ we, int64_t T, int H,
@@ -316,6 +321,17 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[m][e] = make_float2(0.f, 0.f);
+    }
+
+    // the fused weight in fp64 for the dot product (exact: w is an fp32 value)
+    double wd[MAXV][8];
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            wd[m][2 * e] = (double)w[m][e].x;
+            wd[m][2 * e + 1] = (double)w[m][e].y;
+        }
     }
 
     const int64_t G = gridDim.x, first = blockIdx.x;
@@ -353,8 +369,8 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
                     pk2 = __ffma2_rn(kf[e], kf[e], pk2);
                     pg2 = __ffma2_rn(gf[e], vf[e], pg2);
                     const float2 xk = __fmul2_rn(xf[e], kf[e]);   // exact
-                    pa = fma((double)xk.x, (double)w[m][e].x, pa);
-                    pa = fma((double)xk.y, (double)w[m][e].y, pa);
+                    pa = fma((double)xk.x, wd[m][2 * e], pa);
+                    pa = fma((double)xk.y, wd[m][2 * e + 1], pa);
                 }
             }
         }
