@@ -64,6 +64,46 @@ def test_row_widths_and_ragged_shapes(oracle_lib, D):
     np.testing.assert_array_equal(bf16_bits(rows).reshape(want_rows.shape), want_rows)
 
 
+def _random_case(r, L, J, D, B, S, n_max=3, vocab=5000, prime_base=1009):
+    tokens = r.integers(0, vocab, size=(B, S), dtype=np.int64)
+    mult = r.integers(0, 2**64, size=(L, n_max), dtype=np.uint64, endpoint=False) | np.uint64(1)
+    nn = r.integers(1, n_max + 1, size=L).astype(np.int32)
+    sizes = inputs.consecutive_primes(prime_base, L * J).reshape(L, J)
+    tables = inputs.normal_bf16(int(r.integers(1 << 30)), 0, (int(sizes.sum()), D))
+    return dict(tokens=tokens, multipliers=mult, ngram_n=nn, table_sizes=sizes, tables=tables,
+                pad_id=-3)
+
+
+# (L, J, D): from one table of 8-value rows to 32 tables, rows of 16 to 512
+# bytes (one to four 16-byte chunks per lane), n-grams up to order 8
+@pytest.mark.parametrize("L,J,D", [(1, 1, 8), (2, 8, 64), (3, 5, 136), (2, 8, 256), (4, 8, 8),
+                                   (1, 16, 256), (4, 8, 256), (3, 11, 64)])
+def test_gather_paths_bit_exact(oracle_lib, L, J, D):
+    r = np.random.default_rng(L * 1000 + J * 10 + D)
+    h = _random_case(r, L, J, D, B=3, S=37, n_max=8)    # n-grams up to the longest history
+    idx, rows = _run(h)
+    want = oracle_lib.engram_hash(h["tokens"], h["multipliers"], h["ngram_n"], h["table_sizes"],
+                                  pad_id=h["pad_id"])
+    np.testing.assert_array_equal(idx.cpu().numpy(), want)
+    want_rows = oracle_lib.engram_gather(want, h["table_sizes"], h["tables"], D)
+    np.testing.assert_array_equal(bf16_bits(rows).reshape(want_rows.shape), want_rows)
+
+
+@pytest.mark.parametrize("B,S,L,J,D", [(5, 4001, 2, 8, 64), (5, 4001, 2, 8, 136), (4, 30011, 1, 2, 8)])
+def test_many_tokens_per_warp(oracle_lib, B, S, L, J, D):
+    # tens of thousands of tokens, up to 120K: many waves of CTAs, sequences
+    # that span several CTAs' token ranges
+    r = np.random.default_rng(D + S)
+    h = _random_case(r, L, J, D, B=B, S=S)
+    idx, rows = _run(h)
+    want = oracle_lib.engram_hash(h["tokens"], h["multipliers"], h["ngram_n"], h["table_sizes"],
+                                  pad_id=h["pad_id"])
+    np.testing.assert_array_equal(idx.cpu().numpy(), want)
+    want_rows = oracle_lib.engram_gather(want, h["table_sizes"], h["tables"], D)
+    np.testing.assert_array_equal(bf16_bits(rows).reshape(want_rows.shape), want_rows)
+    assert eng.engram_read_device_error() == 0
+
+
 def test_large_table_sizes_and_full_range_ids(oracle_lib):
     # unsigned remainders for table sizes up to 2^62 and ids across all of int64
     import oracle_pins
