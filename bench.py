@@ -601,6 +601,34 @@ def run_gather_bwd_only(args):
                       "us": round(us, 2), "calls": args.steps, "warmup": args.warmup}), flush=True)
 
 
+def run_hash_gather_only(args):
+    """Profiling aid: engram_hash_gather alone on the workload's tokens and
+    tables (no gate tensors on the device: about 2.3 GB at the full-path
+    workload).  Prints one JSON line describing this auxiliary measurement."""
+    import torch
+
+    import engram_conditional_memory_hash_b200 as eng
+    from engram_conditional_memory_hash_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workload(args)
+    h = inputs.hash_inputs(w)
+    tokens = torch.from_numpy(h["tokens"]).to(dev)
+    tables = torch.from_numpy(h["tables"].view(np.int16)).view(torch.bfloat16).to(dev)
+    idx = torch.empty((w.B, w.S, w.L, w.J), dtype=torch.int64, device=dev)
+    rows = torch.empty((w.B, w.S, w.L, w.J, w.D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    us = time_calls(lambda: eng.engram_hash_gather(tokens, h["multipliers"], h["ngram_n"],
+                                                   h["table_sizes"], tables, pad_id=h["pad_id"],
+                                                   idx_out=idx, rows_out=rows, stream=stream),
+                    stream, dev, warmup=args.warmup, calls=args.steps)
+    ab = algorithmic_bytes(w.T, 1, w.L, w.J, w.D, 1)["hash_gather"]
+    print(json.dumps({"part": "hash_gather", "workload": w.name, "T": w.T, "us": round(us, 2),
+                      "algorithmic_bytes": ab, "GB/s": round(ab / (us / 1e6) / 1e9, 1),
+                      "calls": args.steps, "warmup": args.warmup}), flush=True)
+
+
 # ----------------------------------------------------------- reference arm --
 
 def run_reference(args):
@@ -669,14 +697,16 @@ def main():
                     help="tokens per reference-arm step (0: sized from --ref-seconds)")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="CPU time the whole reference-arm run aims at")
-    ap.add_argument("--part", choices=["all", "gather_bwd"], default="all",
-                    help="gather_bwd: time engram_gather_bwd alone (profiling aid)")
+    ap.add_argument("--part", choices=["all", "gather_bwd", "hash_gather"], default="all",
+                    help="gather_bwd / hash_gather: time that call alone (profiling aid)")
     ap.add_argument("--prime-base", type=int, default=0,
                     help="with --part gather_bwd: tables of the primes from this base")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.part == "gather_bwd":
         run_gather_bwd_only(args)
+    elif args.part == "hash_gather":
+        run_hash_gather_only(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -323,6 +323,8 @@ engram_status_t engram_hash_gather(const int64_t *tokens, int64_t B, int64_t S,
         }
     }
     if (T == 0) return ENGRAM_OK;
+    p.inv_L = ~uint64_t(0) / (uint64_t)L;
+    p.inv_S = ~uint64_t(0) / (uint64_t)S;
     if (!tokens) return fail(ENGRAM_ERR_INVALID_ARG, "tokens is NULL");
     if (!aligned(tokens, 8)) return fail(ENGRAM_ERR_INVALID_ARG, "tokens must be 8-byte aligned");
     if (idx_out && !aligned(idx_out, 8)) return fail(ENGRAM_ERR_INVALID_ARG, "idx_out must be 8-byte aligned");

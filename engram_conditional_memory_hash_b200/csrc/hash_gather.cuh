@@ -43,6 +43,7 @@ struct HashParams {
     uint64_t P[kHashMaxTables];              // rows of table q = l*J + j
     uint64_t inv[kHashMaxTables];            // floor((2^64 - 1) / P[q])
     int64_t row0[kHashMaxTables];            // first row of table q in `tables`
+    uint64_t inv_L, inv_S;                   // floor((2^64 - 1) / L), floor((2^64 - 1) / S)
 };
 
 __device__ __forceinline__ uint64_t mod_by_inverse(uint64_t h, uint64_t P, uint64_t inv)
@@ -50,6 +51,20 @@ __device__ __forceinline__ uint64_t mod_by_inverse(uint64_t h, uint64_t P, uint6
     const uint64_t q = __umul64hi(h, inv);
     const uint64_t r = h - q * P;
     return r >= P ? r - P : r;
+}
+
+// Quotient and remainder of x by d >= 1 with the same reciprocal (the integer
+// divisions the kernel needs by the runtime L and S, without a 64-bit divide).
+__device__ __forceinline__ uint64_t div_by_inverse(uint64_t x, uint64_t d, uint64_t inv, uint64_t &rem)
+{
+    uint64_t q = __umul64hi(x, inv);
+    uint64_t r = x - q * d;
+    if (r >= d) {
+        ++q;
+        r -= d;
+    }
+    rem = r;
+    return q;
 }
 
 // CPL: 16-byte chunks per lane per row (rows of up to 64 * CPL bf16 values).
@@ -74,9 +89,11 @@ hash_gather_kernel(const int64_t *__restrict__ tokens, const uint4 *__restrict__
         int l = 0;
         uint64_t h = 0;
         if (active) {
-            const int64_t t = gid / p.L;
-            l = (int)(gid - t * p.L);
-            const int64_t s = t % p.S;
+            uint64_t lr, sr;
+            const int64_t t = (int64_t)div_by_inverse((uint64_t)gid, (uint64_t)p.L, p.inv_L, lr);
+            l = (int)lr;
+            div_by_inverse((uint64_t)t, (uint64_t)p.S, p.inv_S, sr);
+            const int64_t s = (int64_t)sr;
             for (int i = 0; i < p.ngram_n[l]; ++i) {
                 const int64_t tok = (s - i >= 0) ? __ldg(tokens + (t - i)) : p.pad_id;
                 h ^= (uint64_t)tok * p.mult[l][i];
