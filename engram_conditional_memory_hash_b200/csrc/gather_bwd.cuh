@@ -144,8 +144,10 @@ gbwd_mark_kernel(const int64_t *__restrict__ idx, const __grid_constant__ Gather
 // the round's entry l); a round's unique entries are dealt to the warp's
 // 32 / LPR groups of LPR lanes, U at a time per group, lane cv owning the
 // columns [8 cv, 8 cv + 8).
+// Four CTAs per SM (64 registers a thread): more resident warps outweigh the
+// few registers spilled (218 -> 209 us per call at the full-path workload).
 template <int LPR, int U>
-__global__ void __launch_bounds__(kUniqThreads)
+__global__ void __launch_bounds__(kUniqThreads, 4)
 gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_rows,
                    const __grid_constant__ GatherBwdParams p, const uint32_t *__restrict__ dupmap,
                    float4 *__restrict__ d_tables, uint32_t *__restrict__ stage_keys,
@@ -487,9 +489,10 @@ __device__ __forceinline__ void add_bf16x8(double a[8], const uint4 &q)
 // from those registers; a row read several times is summed afterwards (a long
 // run of one hot row by the whole warp, the groups splitting its gradients),
 // so the fp64 accumulators of that case do not add to the registers of the
-// common one.
+// common one.  Four CTAs per SM (64 registers a thread, a few spilled) run
+// faster than three (209 -> 206 us per call at the full-path workload).
 template <int LPR, int U>
-__global__ void __launch_bounds__(kSegThreads, 3)
+__global__ void __launch_bounds__(kSegThreads, 4)
 gbwd_segment_kernel(const uint32_t *__restrict__ keys, const uint32_t *__restrict__ vals,
                     const uint4 *__restrict__ d_rows, const __grid_constant__ GatherBwdParams p,
                     float4 *__restrict__ d_tables, double *__restrict__ carry_a,
