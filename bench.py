@@ -210,6 +210,13 @@ def workload(args):
     return w
 
 
+def gather_bwd_bytes(T: int, L: int, J: int, D: int, unique_rows: int) -> int:
+    """Bytes engram_gather_bwd must move per call: every entry's index (8 B) and
+    bf16 gradient row (2D B) read once, and each of the unique_rows table rows it
+    touches read and written once in fp32 (2 x 4D B)."""
+    return T * L * J * (8 + 2 * D) + unique_rows * 2 * 4 * D
+
+
 def time_calls(call, stream, dev, warmup: int, calls: int) -> float:
     """Microseconds per call of `call` (which enqueues GPU work on `stream`):
     `warmup` calls, then `calls` calls enqueued back to back between two CUDA
@@ -396,7 +403,7 @@ def run_ours(args):
                                                       d_tables, workspace=ws, stream=stream),
                         stream, dev, warmup=3, calls=20)
         # idx read + d_rows read + one read and one write of every touched fp32 table row
-        gb_bytes = T * L * J * (8 + 2 * D) + uniq * 2 * 4 * D
+        gb_bytes = gather_bwd_bytes(T, L, J, D, uniq)
         gbs = gb_bytes / (us / 1e6) / 1e9
         gbwd = {"us": round(us, 2), "algorithmic_bytes": gb_bytes, "GB/s": round(gbs, 1),
                 "frac": round(gbs / peak, 4), "traffic": committed_traffic("gather_bwd", T),

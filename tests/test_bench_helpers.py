@@ -19,6 +19,16 @@ def test_algorithmic_bytes_full_path():
     assert ab["grad_w_reduce"] == G * 4 * H + 8 * H + 4 * H
 
 
+def test_gather_bwd_bytes():
+    # full path: 1,048,576 entries (8 B index + 128 B gradient row each) and
+    # 821,830 distinct table rows (256 B fp32, read and written)
+    assert bench.gather_bwd_bytes(65536, 2, 8, 64, 821830) == 1048576 * 136 + 821830 * 512 \
+        == 563383296
+    # no entries, nothing to move; one row read by every entry is read and written once
+    assert bench.gather_bwd_bytes(0, 2, 8, 64, 0) == 0
+    assert bench.gather_bwd_bytes(10, 1, 1, 8, 1) == 10 * 24 + 64
+
+
 def test_every_kernel_has_sources_and_a_digest():
     for k in ("hash_gather", "gate_fwd", "gate_bwd", "grad_w_reduce", "gather_bwd"):
         d = bench.source_digest(k)
