@@ -10,6 +10,20 @@ for _p in (ROOT, TESTS):
         sys.path.insert(0, _p)
 
 
+def pytest_sessionstart(session):
+    # Bring the CUDA library and the CPU oracle up to date with their sources
+    # (make does nothing when they are current).  nvcc cross-compiles for
+    # sm_100a without a GPU, so this works on CPU-only machines too.
+    import shutil
+    import subprocess
+    if shutil.which("make") is None:
+        return
+    for d in (os.path.join(ROOT, "engram_conditional_memory_hash_b200", "csrc"), os.path.join(ROOT, "oracle")):
+        r = subprocess.run(["make", "-s", "-C", d], capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"building {d} failed:\n{r.stdout}\n{r.stderr}")
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size case, minutes of CPU time")
