@@ -3,8 +3,10 @@
 
 One step = one pass of the whole path over one batch of synthetic input:
 engram_hash_gather (n-gram hash + gather of 16 table rows per token),
-engram_gate_fwd, engram_gate_bwd and engram_grad_w_reduce (and, on more than
-one GPU, an NCCL all-reduce of dwh/dwe, the path's one exchange step).
+engram_gate_fwd and engram_gate_bwd_fused (the gate backward with the
+weight-gradient reduction in the same kernel) -- three launches -- and, on
+more than one GPU, an all-reduce of dwh/dwe, the path's one exchange step
+(NCCL by default; --dist-backend gloo runs the same step over gloo).
 
 Default workload ("full_path"): 4 x 16384 = 65536 tokens with Zipf(1.1) ids
 over a 129280-id vocabulary, 2 n-gram layers (2-, 3-grams) x 8 tables of
@@ -14,8 +16,12 @@ L2 (each gate tensor is 940 MB), so no L2 flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Prints one JSON line (rank 0).  With --impl reference the fp64 CPU oracle is
-timed instead, on a bounded sample of tokens per step.
+Prints one JSON line (rank 0).  After the default workload the same process
+measures the other workloads (tiny, gate_fwd, gate_fwdbwd, hash_gather) and
+reports them under "configs".  Every "frac" is a fraction of the measured
+copy bandwidth (MEASURED_PEAKS.json hbm_gbs); every "frac_nominal" a fraction
+of the nominal 8 TB/s HBM3e bandwidth.  With --impl reference the fp64 CPU
+oracle is timed instead, on a bounded sample of tokens per step.
 """
 from __future__ import annotations
 
@@ -37,6 +43,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Engram gate fwd+bwd tokens/s and HBM GB/s (% of B200 peak) at H=7168"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0     # the ~8 TB/s of B200 HBM3e the targets are stated against
+BAR_FRACTION = 0.7           # target: every kernel at >= 70% of the nominal bandwidth
+L2_FLUSH_BYTES = 2 * 126 * 1024 * 1024
 _CSRC = "engram_conditional_memory_hash_b200/csrc/"
 # the sources that define each kernel and its launch (a change to any of them
 # makes the committed DRAM counters of that kernel stale)
@@ -44,7 +53,6 @@ KERNEL_SOURCES = {
     "hash_gather": ["hash_gather.cuh", "common.cuh", "engram_abi.cu"],
     "gate_fwd": ["gate_kernels.cuh", "common.cuh", "engram_abi.cu"],
     "gate_bwd": ["gate_kernels.cuh", "common.cuh", "engram_abi.cu"],
-    "grad_w_reduce": ["gate_kernels.cuh", "common.cuh", "engram_abi.cu"],
     "gather_bwd": ["gather_bwd.cuh", "gather_bwd_abi.inl", "hash_gather.cuh", "common.cuh"],
 }
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -54,18 +62,29 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 def algorithmic_bytes(T: int, H: int, L: int, J: int, D: int, G: int) -> dict:
     """Bytes each kernel must move per launch (the minimum: every input read
-    once, every output written once; table rows counted per gathered row)."""
+    once, every output written once; table rows counted per gathered row).
+    gate_bwd is the fused backward: its own bytes plus the reduction's
+    (partial rows written and read back, dwh and dwe written)."""
     rows = T * L * J
+    reduce = G * 4 * H + 2 * 4 * H + 2 * 2 * H
     return {
         # tokens read + idx written + rows read + rows written
         "hash_gather": T * 8 + rows * 8 + 2 * rows * D * 2,
         # x, k, v read; out written; gate written; wh, we read
         "gate_fwd": T * (4 * 2 * H + 4) + 2 * 2 * H,
-        # g, x, k, v read; dx, dk, dv written; partial rows written; wh, we read
-        "gate_bwd": T * 7 * 2 * H + G * 4 * H + 2 * 2 * H,
-        # partial rows read; dwh, dwe written; wh, we read
-        "grad_w_reduce": G * 4 * H + 2 * 4 * H + 2 * 2 * H,
+        # g, x, k, v read; dx, dk, dv written; partial rows written; wh, we
+        # read; then the reduction of the partial rows
+        "gate_bwd": T * 7 * 2 * H + G * 4 * H + 2 * 2 * H + reduce,
     }
+
+
+def kernel_entry(us: float, nbytes: int, peak: float) -> dict:
+    """Time, algorithmic bandwidth and its fractions of the measured and the
+    nominal peak for one launch; us_at_bar is the time at 70% of nominal."""
+    gbs = nbytes / (us / 1e6) / 1e9
+    return {"us": round(us, 2), "algorithmic_bytes": int(nbytes), "GB/s": round(gbs, 1),
+            "frac": round(gbs / peak, 4), "frac_nominal": round(gbs / NOMINAL_HBM_GBS, 4),
+            "us_at_bar": round(nbytes / (BAR_FRACTION * NOMINAL_HBM_GBS * 1e9) * 1e6, 2)}
 
 
 def source_digest(kernel: str) -> str:
@@ -118,7 +137,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.idx)],
+                 "-lms", "20", "-i", str(self.idx)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -202,6 +221,8 @@ def workload(args):
     sequences where possible; used for small profiling runs)."""
     from engram_conditional_memory_hash_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
+    if getattr(args, "hidden", 0):
+        w = dataclasses.replace(w, H=args.hidden)
     if args.tokens and args.tokens < w.T:
         if args.tokens >= w.S:
             w = dataclasses.replace(w, B=args.tokens // w.S)
@@ -248,14 +269,14 @@ def run_ours(args):
     import torch.distributed as dist
 
     import engram_conditional_memory_hash_b200 as eng
-    from engram_conditional_memory_hash_b200 import dp, inputs
+    from engram_conditional_memory_hash_b200 import step as engram_step
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        kw = {"device_id": dev} if args.dist_backend == "nccl" else {}
+        dist.init_process_group(args.dist_backend, timeout=datetime.timedelta(seconds=120), **kw)
     w = workload(args)
     T, H, L, J, D = w.T, w.H, w.L, w.J, w.D
 
@@ -266,57 +287,24 @@ def run_ours(args):
     def to_dev(a):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
 
-    tables = torch.from_numpy(hin["tables"].view(np.int16)).view(torch.bfloat16).to(dev)
-    wh = to_dev(gin["wh"])
-    we = to_dev(gin["we"])
-    G = eng.engram_gate_bwd_num_partials(T, H)
+    tables = to_dev(hin["tables"]).view(-1, D)
+    st = engram_step.EngramStep(w.B, w.S, H, dev, tables, to_dev(gin["wh"]), to_dev(gin["we"]),
+                                hin["multipliers"], hin["ngram_n"], hin["table_sizes"],
+                                pad_id=hin["pad_id"], eps=w.eps)
+    G = st.G
 
-    def make_buffers(fill: bool):
-        """One set of per-step device buffers (inputs filled from the host when asked)."""
-        b = {"tokens": torch.empty((w.B, w.S), dtype=torch.int64, device=dev)}
+    def fill(b):
+        b.tokens.copy_(torch.from_numpy(hin["tokens"]))
         for n in ("x", "k", "v", "g"):
-            b[n] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-        if fill:
-            b["tokens"].copy_(torch.from_numpy(hin["tokens"]))
-            for n in ("x", "k", "v", "g"):
-                b[n].copy_(torch.from_numpy(gin[n].view(np.int16)).view(torch.bfloat16))
-        b["idx"] = torch.empty((w.B, w.S, L, J), dtype=torch.int64, device=dev)
-        b["rows"] = torch.empty((w.B, w.S, L, J, D), dtype=torch.bfloat16, device=dev)
-        b["out"] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-        b["gate"] = torch.empty((T,), dtype=torch.float32, device=dev)
-        for n in ("dx", "dk", "dv"):
-            b[n] = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-        b["part"] = torch.empty((G, H), dtype=torch.float32, device=dev)
-        b["dw"] = torch.empty((2, H), dtype=torch.float32, device=dev)
+            getattr(b, n).copy_(torch.from_numpy(gin[n].view(np.int16)).view(torch.bfloat16))
         return b
 
-    buf0 = make_buffers(True)
+    buf0 = fill(st.buffers())
     stream = torch.cuda.current_stream(dev)
-    names = ["hash_gather", "gate_fwd", "gate_bwd", "grad_w_reduce"]
-
-    def step(b=buf0, ev=None, s=stream):
-        def mark(i):
-            if ev is not None:
-                ev[i].record(s)
-        mark(0)
-        eng.engram_hash_gather(b["tokens"], hin["multipliers"], hin["ngram_n"],
-                               hin["table_sizes"], tables, pad_id=hin["pad_id"],
-                               idx_out=b["idx"], rows_out=b["rows"], stream=s)
-        mark(1)
-        eng.engram_gate_fwd(b["x"], b["k"], b["v"], wh, we, eps=w.eps, out=b["out"],
-                            gate=b["gate"], stream=s)
-        mark(2)
-        eng.engram_gate_bwd(b["g"], b["x"], b["k"], b["v"], wh, we, eps=w.eps, dx=b["dx"],
-                            dk=b["dk"], dv=b["dv"], w_partial=b["part"], stream=s)
-        mark(3)
-        eng.engram_grad_w_reduce(b["part"], wh, we, dwh=b["dw"][0], dwe=b["dw"][1], stream=s)
-        mark(4)
-        if world > 1:
-            with torch.cuda.stream(s):
-                dp.allreduce_weight_grads(b["dw"])
+    names = list(engram_step.LAUNCHES)
 
     for _ in range(args.warmup):
-        step()
+        st.run(buf0, stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -324,7 +312,8 @@ def run_ours(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+           for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -333,7 +322,7 @@ def run_ours(args):
     wall0 = time.time()
     start.record(stream)
     for i in range(args.steps):
-        step(ev=evs[i])
+        st.run(buf0, stream, events=evs[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
     wall1 = time.time()
@@ -360,10 +349,10 @@ def run_ours(args):
     if args.uniform_control and rank == 0 and w.vocab > 0:
         from engram_conditional_memory_hash_b200 import inputs as _inp
         utok = torch.from_numpy(_inp.uniform_ids(w.seed, 99, (w.B, w.S), 0, w.vocab)).to(dev)
-        flush = torch.empty(2 * 126 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
         # its own outputs: the step's indices in buf0 stay those of the step's
         # tokens (the gather backward below runs on them)
-        uidx, urows = torch.empty_like(buf0["idx"]), torch.empty_like(buf0["rows"])
+        uidx, urows = torch.empty_like(buf0.idx), torch.empty_like(buf0.rows)
         ts = []
         for it in range(13):
             flush.zero_()
@@ -376,17 +365,15 @@ def run_ours(args):
             torch.cuda.synchronize(dev)
             if it >= 3:
                 ts.append(e0.elapsed_time(e1))
-        us = float(np.median(ts)) * 1e3
-        gbs = ab["hash_gather"] / (us / 1e6) / 1e9
-        uniform = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4),
-                   "ids": f"uniform over [0, {w.vocab}), L2 flushed before each launch"}
+        uniform = kernel_entry(float(np.median(ts)) * 1e3, ab["hash_gather"], peak)
+        uniform["ids"] = f"uniform over [0, {w.vocab}), L2 flushed before each launch"
         del flush, uidx, urows
 
     # Gather backward (the transpose of the gather: row gradients summed into
-    # the fp32 table gradient), timed on its own: it is not one of the four
-    # calls of the step.  d_rows is a synthetic N(0,1) gradient of the gathered
-    # rows; d_tables (4.1 GB) accumulates across iterations, which does not
-    # change the work.
+    # the fp32 table gradient), timed on its own: it is not one of the calls of
+    # the step.  d_rows is a synthetic N(0,1) gradient of the gathered rows;
+    # d_tables (4.1 GB) accumulates across iterations, which does not change
+    # the work.
     gbwd = None
     if args.gather_bwd and rank == 0 and w.has_hash:
         from engram_conditional_memory_hash_b200 import inputs as _inp
@@ -398,29 +385,23 @@ def run_ours(args):
                          device=dev)
         first = torch.from_numpy(np.concatenate(
             [[0], np.cumsum(hin["table_sizes"].ravel())[:-1]])).to(dev)
-        uniq = int(torch.unique(buf0["idx"].view(T, L * J) + first[None]).numel())
-        us = time_calls(lambda: eng.engram_gather_bwd(buf0["idx"], hin["table_sizes"], d_rows,
+        uniq = int(torch.unique(buf0.idx.view(T, L * J) + first[None]).numel())
+        us = time_calls(lambda: eng.engram_gather_bwd(buf0.idx, hin["table_sizes"], d_rows,
                                                       d_tables, workspace=ws, stream=stream),
                         stream, dev, warmup=3, calls=20)
         # idx read + d_rows read + one read and one write of every touched fp32 table row
-        gb_bytes = gather_bwd_bytes(T, L, J, D, uniq)
-        gbs = gb_bytes / (us / 1e6) / 1e9
-        gbwd = {"us": round(us, 2), "algorithmic_bytes": gb_bytes, "GB/s": round(gbs, 1),
-                "frac": round(gbs / peak, 4), "traffic": committed_traffic("gather_bwd", T),
-                "unique_rows": uniq, "entries": T * L * J,
-                "launches": 12,
-                "what": "engram_gather_bwd on the step's indices: rows read once updated in "
-                        "place, the rest listed, radix-sorted by row and summed in fp64; fp32 "
-                        "table-gradient update; 20 calls back to back, CUDA events around "
-                        "them"}
+        gbwd = kernel_entry(us, gather_bwd_bytes(T, L, J, D, uniq), peak)
+        gbwd.update({"traffic": committed_traffic("gather_bwd", T), "unique_rows": uniq,
+                     "entries": T * L * J, "launches": GATHER_BWD_LAUNCHES,
+                     "what": "engram_gather_bwd on the step's indices: rows read once updated "
+                             "in place, the rest listed, radix-sorted by row and summed in fp64; "
+                             "fp32 table-gradient update; 20 calls back to back, CUDA events "
+                             "around them"})
         del d_rows, d_tables, ws
 
-    kern = {}
-    for n in names:
-        us = per_kernel_ms[n] * 1e3
-        gbs = ab[n] / (per_kernel_ms[n] / 1e3) / 1e9
-        kern[n] = {"us": round(us, 2), "algorithmic_bytes": ab[n], "GB/s": round(gbs, 1),
-                   "frac": round(gbs / peak, 4)}
+    kern = {n: kernel_entry(per_kernel_ms[n] * 1e3, ab[n], peak) for n in names}
+    kern["gate_bwd"]["what"] = ("engram_gate_bwd_fused: backward and weight-gradient reduction "
+                                "in one kernel")
     step_bytes = sum(ab.values())
     dominant = max(names, key=lambda n: per_kernel_ms[n])
     roof = {
@@ -430,8 +411,10 @@ def run_ours(args):
         "peak": peak,
         "unit": "GB/s",
         "frac": kern[dominant]["frac"],
-        "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-        else "fallback 6650 GB/s",
+        "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, a copy-kernel bandwidth)"
+        if peak_kind == "measured" else "fallback 6650 GB/s",
+        "frac_nominal": kern[dominant]["frac_nominal"],
+        "peak_nominal": NOMINAL_HBM_GBS,
         "traffic": committed_traffic(dominant, T),
     }
 
@@ -439,17 +422,16 @@ def run_ours(args):
     e2e = None
     if args.e2e_steps > 0:
         # Host buffers in and out: pinned host inputs are uploaded on a copy
-        # stream, the four C-ABI calls run on the compute stream, every output
+        # stream, the step's C-ABI calls run on the compute stream, every output
         # is downloaded on a second copy stream.  Two device buffer sets let the
         # upload of step i+1 and the download of step i-1 overlap step i.
-        in_names = ("tokens", "x", "k", "v", "g")
-        out_names = ("idx", "rows", "out", "gate", "dx", "dk", "dv", "dw")
+        in_names, out_names = engram_step.StepBuffers.INPUTS, engram_step.StepBuffers.OUTPUTS
         host_in = {"tokens": torch.from_numpy(hin["tokens"]).pin_memory()}
         for n in ("x", "k", "v", "g"):
             host_in[n] = torch.from_numpy(gin[n].view(np.int16)).view(torch.bfloat16).pin_memory()
-        host_out = {n: torch.empty(buf0[n].shape, dtype=buf0[n].dtype, pin_memory=True)
-                    for n in out_names}
-        bufs = [buf0, make_buffers(False)]
+        host_out = {n: torch.empty(getattr(buf0, n).shape, dtype=getattr(buf0, n).dtype,
+                                   pin_memory=True) for n in out_names}
+        bufs = [buf0, st.buffers()]
         h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         comp_s = stream
         ev_h2d = [torch.cuda.Event() for _ in range(2)]
@@ -465,17 +447,17 @@ def run_ours(args):
                 if i >= 2:
                     h2d_s.wait_event(ev_comp[bi])        # inputs of step i-2 consumed
                 for n in in_names:
-                    b[n].copy_(host_in[n], non_blocking=True)
+                    getattr(b, n).copy_(host_in[n], non_blocking=True)
                 ev_h2d[bi].record(h2d_s)
             comp_s.wait_event(ev_h2d[bi])
             if i >= 2:
                 comp_s.wait_event(ev_d2h[bi])            # outputs of step i-2 downloaded
-            step(b, s=comp_s)
+            st.run(b, comp_s)
             ev_comp[bi].record(comp_s)
             with torch.cuda.stream(d2h_s):
                 d2h_s.wait_event(ev_comp[bi])
                 for n in out_names:
-                    host_out[n].copy_(b[n], non_blocking=True)
+                    host_out[n].copy_(getattr(b, n), non_blocking=True)
                 ev_d2h[bi].record(d2h_s)
 
         for i in range(2):                                # warm-up
@@ -498,9 +480,19 @@ def run_ours(args):
         e2e = {"value": round(world * T / (e_ms / args.e2e_steps / 1e3), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps,
-               "path": "pinned host inputs -> H2D (copy stream) -> the four C-ABI calls -> D2H "
-                       "of every output (second copy stream); two device buffer sets overlap "
-                       "step i's compute with the neighbouring steps' copies"}
+               "path": "pinned host inputs -> H2D (copy stream) -> the step's three C-ABI calls "
+                       "-> D2H of every output (second copy stream); two device buffer sets "
+                       "overlap step i's compute with the neighbouring steps' copies"}
+        del bufs, host_in, host_out
+    del buf0, st, tables
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads, one GPU, same process (rank 0 only) -----------
+    configs = None
+    if args.configs and rank == 0:
+        configs = {name: measure_config(name, dev, peak)
+                   for name in ("tiny", "gate_fwd", "gate_fwdbwd", "hash_gather")}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) -------
     cpu = None
@@ -549,26 +541,110 @@ def run_ours(args):
                             f"~1M rows x {D} bf16, gate fwd+bwd at H={H}",
                 "T": T, "H": H, "L": L, "J": J, "D": D, "G": G,
                 "l2": "inputs larger than L2 (940 MB per gate tensor, 2.05 GB tables); no flush",
-                "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                "parallelism": f"dp{world} ({args.dist_backend})" if world > 1 else "single GPU",
             },
             "hbm_gbs": round(step_bytes / (ms_per_step / 1e3) / 1e9, 1),
             "hbm_frac": round(step_bytes / (ms_per_step / 1e3) / 1e9 / peak, 4),
+            "hbm_frac_nominal": round(step_bytes / (ms_per_step / 1e3) / 1e9 / NOMINAL_HBM_GBS, 4),
+            "peaks": {"frac": f"of the measured copy bandwidth, {peak} GB/s ({peak_kind})",
+                      "frac_nominal": f"of the nominal {NOMINAL_HBM_GBS:.0f} GB/s",
+                      "us_at_bar": f"time at {BAR_FRACTION:.0%} of the nominal bandwidth"},
             "gate_fwd_bwd_tokens_per_s": round(
-                world * T / ((per_kernel_ms["gate_fwd"] + per_kernel_ms["gate_bwd"]
-                              + per_kernel_ms["grad_w_reduce"]) / 1e3), 1),
+                world * T / ((per_kernel_ms["gate_fwd"] + per_kernel_ms["gate_bwd"]) / 1e3), 1),
             "kernels": kern,
             "hash_gather_uniform_ids": uniform,
             "gather_bwd": gbwd,
+            "configs": configs,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": len(names) * args.steps,
             "clocks": clk,
             "input_generation_s": round(t_gen, 1),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+GATHER_BWD_LAUNCHES = 12
+
+
+def measure_config(name: str, dev, peak: float, iters: int = 20, warmup: int = 3) -> dict:
+    """Time the named workload's own calls on one GPU: per launch, the median
+    over `iters` iterations of CUDA events around it (after `warmup`).
+    Workloads whose inputs fit in L2 (tiny, hash_gather's hot rows) get an L2
+    flush before every iteration; the gate workloads' inputs are larger than
+    L2 and run back to back."""
+    import torch
+
+    import engram_conditional_memory_hash_b200 as eng
+    from engram_conditional_memory_hash_b200 import inputs
+    from engram_conditional_memory_hash_b200 import step as engram_step
+
+    w = inputs.WORKLOADS[name]
+    stream = torch.cuda.current_stream(dev)
+    T = w.T
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    calls = {}           # launch name -> callable enqueuing it
+    H = w.H
+    G = 1
+    if w.has_hash:
+        h = inputs.hash_inputs(w)
+        tokens = torch.from_numpy(h["tokens"]).to(dev)
+        tables = bf(h["tables"]).view(-1, w.D)
+        idx = torch.empty((w.B, w.S, w.L, w.J), dtype=torch.int64, device=dev)
+        rows = torch.empty((w.B, w.S, w.L, w.J, w.D), dtype=torch.bfloat16, device=dev)
+        calls["hash_gather"] = lambda: eng.engram_hash_gather(
+            tokens, h["multipliers"], h["ngram_n"], h["table_sizes"], tables, pad_id=h["pad_id"],
+            idx_out=idx, rows_out=rows, stream=stream)
+    if w.has_gate:
+        gi = {n: bf(a) for n, a in inputs.gate_inputs(w).items()}
+        out = torch.empty_like(gi["x"])
+        gate = torch.empty((T,), dtype=torch.float32, device=dev)
+        calls["gate_fwd"] = lambda: eng.engram_gate_fwd(
+            gi["x"], gi["k"], gi["v"], gi["wh"], gi["we"], eps=w.eps, out=out, gate=gate,
+            stream=stream)
+        if w.backward:
+            G = eng.engram_gate_bwd_num_partials(T, H)
+            dx, dk, dv = (torch.empty_like(gi["x"]) for _ in range(3))
+            part = torch.empty((G, H), dtype=torch.float32, device=dev)
+            tickets = torch.zeros((eng.GATE_BWD_TICKETS,), dtype=torch.int32, device=dev)
+            dw = torch.empty((2, H), dtype=torch.float32, device=dev)
+            calls["gate_bwd"] = lambda: eng.engram_gate_bwd_fused(
+                gi["g"], gi["x"], gi["k"], gi["v"], gi["wh"], gi["we"], eps=w.eps, dx=dx, dk=dk,
+                dv=dv, w_partial=part, tickets=tickets, dwh=dw[0], dwe=dw[1], stream=stream)
+    names = [n for n in engram_step.LAUNCHES if n in calls]
+    flush_l2 = name in ("tiny", "hash_gather")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush_l2 else None
+    times = {n: [] for n in names}
+    for it in range(warmup + iters):
+        if flush is not None:
+            flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        ev[0].record(stream)
+        for i, n in enumerate(names):
+            calls[n]()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        if it >= warmup:
+            for i, n in enumerate(names):
+                times[n].append(ev[i].elapsed_time(ev[i + 1]))
+    assert eng.engram_read_device_error() == 0
+    ab = algorithmic_bytes(T, max(H, 1), w.L, w.J, w.D, G)
+    kern = {n: kernel_entry(float(np.median(times[n])) * 1e3, ab[n], peak) for n in names}
+    total_us = sum(k["us"] for k in kern.values())
+    res = {"T": T, "H": H or None, "launches": names, "kernels": kern,
+           "tokens_per_s": round(T / (total_us / 1e6), 1),
+           "l2": "flushed before every iteration" if flush_l2 else
+                 "inputs larger than L2; iterations back to back",
+           "timing": f"median of {iters} iterations after {warmup}, CUDA events per launch"}
+    if w.has_hash:
+        res["tables"] = f"{w.L * w.J} x ~{w.prime_base} rows x {w.D} bf16, ids {w.ids}"
+    return res
 
 
 # ------------------------------------------- gather backward on its own --
@@ -633,6 +709,50 @@ def run_hash_gather_only(args):
     ab = algorithmic_bytes(w.T, 1, w.L, w.J, w.D, 1)["hash_gather"]
     print(json.dumps({"part": "hash_gather", "workload": w.name, "T": w.T, "us": round(us, 2),
                       "algorithmic_bytes": ab, "GB/s": round(ab / (us / 1e6) / 1e9, 1),
+                      "calls": args.steps, "warmup": args.warmup}), flush=True)
+
+
+def run_gate_only(args):
+    """Profiling aid: engram_gate_fwd and engram_gate_bwd_fused alone on the
+    workload's gate tensors (no tables on the device; with --tokens 8192 at
+    H = 7168 about 1 GB).  Prints one JSON line describing this auxiliary
+    measurement."""
+    import torch
+
+    import engram_conditional_memory_hash_b200 as eng
+    from engram_conditional_memory_hash_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workload(args)
+    T, H = w.T, w.H
+    gi = {n: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+          for n, a in inputs.gate_inputs(w).items()}
+    G = eng.engram_gate_bwd_num_partials(T, H)
+    out, dx, dk, dv = (torch.empty_like(gi["x"]) for _ in range(4))
+    gate = torch.empty((T,), dtype=torch.float32, device=dev)
+    part = torch.empty((G, H), dtype=torch.float32, device=dev)
+    tickets = torch.zeros((eng.GATE_BWD_TICKETS,), dtype=torch.int32, device=dev)
+    dw = torch.empty((2, H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        eng.engram_gate_fwd(gi["x"], gi["k"], gi["v"], gi["wh"], gi["we"], eps=w.eps, out=out,
+                            gate=gate, stream=stream)
+
+    def bwd():
+        eng.engram_gate_bwd_fused(gi["g"], gi["x"], gi["k"], gi["v"], gi["wh"], gi["we"],
+                                  eps=w.eps, dx=dx, dk=dk, dv=dv, w_partial=part,
+                                  tickets=tickets, dwh=dw[0], dwe=dw[1], stream=stream)
+
+    us_f = time_calls(fwd, stream, dev, warmup=args.warmup, calls=args.steps)
+    us_b = time_calls(bwd, stream, dev, warmup=args.warmup, calls=args.steps)
+    assert eng.engram_read_device_error() == 0
+    ab = algorithmic_bytes(T, H, 1, 1, 8, G)
+    peak, _ = measured_peak()
+    print(json.dumps({"part": "gate", "workload": w.name, "T": T, "H": H, "G": G,
+                      "gate_fwd": kernel_entry(us_f, ab["gate_fwd"], peak),
+                      "gate_bwd": kernel_entry(us_b, ab["gate_bwd"], peak),
                       "calls": args.steps, "warmup": args.warmup}), flush=True)
 
 
@@ -704,8 +824,15 @@ def main():
                     help="tokens per reference-arm step (0: sized from --ref-seconds)")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="CPU time the whole reference-arm run aims at")
-    ap.add_argument("--part", choices=["all", "gather_bwd", "hash_gather"], default="all",
-                    help="gather_bwd / hash_gather: time that call alone (profiling aid)")
+    ap.add_argument("--part", choices=["all", "gather_bwd", "hash_gather", "gate"], default="all",
+                    help="gather_bwd / hash_gather / gate (forward and fused backward): time "
+                         "those calls alone (profiling aid)")
+    ap.add_argument("--hidden", type=int, default=0,
+                    help="with --part gate: another hidden size (e.g. one the generic kernels take)")
+    ap.add_argument("--dist-backend", choices=["nccl", "gloo"], default="nccl",
+                    help="process-group backend of the multi-GPU all-reduce")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the measurements of the other workloads")
     ap.add_argument("--prime-base", type=int, default=0,
                     help="with --part gather_bwd: tables of the primes from this base")
     args = ap.parse_args()
@@ -714,6 +841,8 @@ def main():
         run_gather_bwd_only(args)
     elif args.part == "hash_gather":
         run_hash_gather_only(args)
+    elif args.part == "gate":
+        run_gate_only(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

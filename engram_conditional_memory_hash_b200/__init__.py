@@ -29,7 +29,8 @@ __all__ = [
     "engram_hash_gather", "engram_gate_fwd", "engram_gate_bwd_num_partials",
     "engram_gate_bwd", "engram_grad_w_reduce", "engram_read_device_error",
     "engram_gate_bwd_noalloc", "engram_gather_bwd_workspace_size", "engram_gather_bwd",
-    "default_scalar", "DEVICE_ERR_PIPELINE_TIMEOUT", "DEVICE_ERR_INDEX_RANGE",
+    "engram_gate_bwd_fused", "GATE_BWD_TICKETS", "default_scalar",
+    "DEVICE_ERR_PIPELINE_TIMEOUT", "DEVICE_ERR_INDEX_RANGE",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,11 +38,14 @@ LIBRARY_NAME = "libengram_b200.so"
 EXPORTED = ("engram_abi_version", "engram_status_string", "engram_last_error",
             "engram_hash_gather", "engram_gate_fwd", "engram_gate_bwd_num_partials",
             "engram_gate_bwd", "engram_grad_w_reduce", "engram_read_device_error",
-            "engram_gate_bwd_noalloc", "engram_gather_bwd_workspace_size", "engram_gather_bwd")
+            "engram_gate_bwd_noalloc", "engram_gather_bwd_workspace_size", "engram_gather_bwd",
+            "engram_gate_bwd_fused")
 
 # codes of the kernels' device error word (engram_read_device_error)
 DEVICE_ERR_PIPELINE_TIMEOUT = 1
 DEVICE_ERR_INDEX_RANGE = 2
+# words of the ticket array of engram_gate_bwd_fused (ENGRAM_GATE_BWD_TICKETS)
+GATE_BWD_TICKETS = 64
 
 
 class EngramError(RuntimeError):
@@ -93,6 +97,9 @@ def lib() -> ctypes.CDLL:
             L.engram_gate_bwd.restype = ctypes.c_int
             L.engram_gate_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _f32, _f32,
                                           _vp, _vp, _vp, _vp, _i64, _vp]
+            L.engram_gate_bwd_fused.restype = ctypes.c_int
+            L.engram_gate_bwd_fused.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _f32, _f32,
+                                                _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
             L.engram_grad_w_reduce.restype = ctypes.c_int
             L.engram_grad_w_reduce.argtypes = [_vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp]
             L.engram_gate_bwd_noalloc.restype = ctypes.c_int
@@ -330,6 +337,67 @@ def engram_gate_bwd(grad_out, x, k, v, wh, we, eps: float = 1e-6, scalar: float 
                                _stream_ptr(stream))
     _check("engram_gate_bwd", st)
     return dx, dk, dv, w_partial
+
+
+_tickets = {}
+
+
+def _stream_tickets(device: torch.device, stream_ptr: int) -> torch.Tensor:
+    """The zeroed ticket array engram_gate_bwd_fused uses for calls on one
+    stream of one device (calls in stream order may share it; the kernel
+    leaves it zero)."""
+    key = (device.index, stream_ptr)
+    t = _tickets.get(key)
+    if t is None:
+        t = torch.zeros((GATE_BWD_TICKETS,), dtype=torch.int32, device=device)
+        _tickets[key] = t
+    return t
+
+
+def engram_gate_bwd_fused(grad_out, x, k, v, wh, we, eps: float = 1e-6,
+                          scalar: float | None = None, *, dx=None, dk=None, dv=None,
+                          w_partial=None, G: int | None = None, tickets=None, dwh=None, dwe=None,
+                          stream=None):
+    """Gate backward with the weight-gradient reduction fused into its tail
+    (one launch for the tuned shapes).  w_partial [G, H] fp32 is scratch;
+    tickets is an int32 [GATE_BWD_TICKETS] device array that is zero before the
+    call and zero after it (one per stream is kept here when None).
+    Returns (dx, dk, dv bf16 [T, H], dwh, dwe fp32 [H])."""
+    T, H = _gate_shapes(x, k, v, wh, we)
+    if tuple(grad_out.shape) != (T, H):
+        raise ValueError("grad_out must be [T, H]")
+    ptrs = [_dev(t, n, torch.bfloat16) for t, n in ((grad_out, "grad_out"), (x, "x"), (k, "k"),
+                                                    (v, "v"), (wh, "wh"), (we, "we"))]
+    if w_partial is not None:
+        if w_partial.dim() != 2 or w_partial.shape[1] != H:
+            raise ValueError("w_partial must be [G, H]")
+        if G is not None and G != w_partial.shape[0]:
+            raise ValueError("G does not match w_partial")
+        G = w_partial.shape[0]
+    if G is None:
+        G = engram_gate_bwd_num_partials(T, H)
+    if w_partial is None:
+        w_partial = torch.empty((G, H), dtype=torch.float32, device=x.device)
+    sp = _stream_ptr(stream)
+    if tickets is None:
+        tickets = _stream_tickets(x.device, sp)
+    if tickets.numel() < GATE_BWD_TICKETS:
+        raise ValueError(f"tickets must hold {GATE_BWD_TICKETS} words")
+    dx = torch.empty_like(x) if dx is None else dx
+    dk = torch.empty_like(x) if dk is None else dk
+    dv = torch.empty_like(x) if dv is None else dv
+    dwh = torch.empty((H,), dtype=torch.float32, device=x.device) if dwh is None else dwh
+    dwe = torch.empty((H,), dtype=torch.float32, device=x.device) if dwe is None else dwe
+    outs = [_dev(t, n, torch.bfloat16) for t, n in ((dx, "dx"), (dk, "dk"), (dv, "dv"))]
+    if scalar is None:
+        scalar = default_scalar(H)
+    st = lib().engram_gate_bwd_fused(*ptrs, T, H, float(eps), float(scalar), *outs,
+                                     _dev(w_partial, "w_partial", torch.float32), int(G),
+                                     _dev(tickets, "tickets", torch.int32),
+                                     _dev(dwh, "dwh", torch.float32),
+                                     _dev(dwe, "dwe", torch.float32), sp)
+    _check("engram_gate_bwd_fused", st)
+    return dx, dk, dv, dwh, dwe
 
 
 def engram_grad_w_reduce(w_partial, wh, we, *, dwh=None, dwe=None, stream=None):

@@ -5,7 +5,8 @@ The Engram section of the page "DeepSeek 开源 TileKernels" (zhichai.net/topic/
 ``torch.autograd.Function`` wrapper around the gate kernels with forward,
 backward and weight-gradient reduction.  ``EngramGateFunction`` is that wrapper
 over this library's C ABI: forward = engram_gate_fwd; backward =
-engram_gate_bwd followed by engram_grad_w_reduce.  ``EngramGate`` is an
+engram_gate_bwd_fused (the backward with engram_grad_w_reduce's reduction in
+its tail, bitwise the same as the two calls).  ``EngramGate`` is an
 ``nn.Module`` holding the two RMSNorm weights.
 
 ``EngramHashGatherFunction`` does the same for the n-gram hash and table-row
@@ -22,8 +23,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (default_scalar, engram_gate_bwd, engram_gate_fwd, engram_gather_bwd,
-               engram_grad_w_reduce, engram_hash_gather)
+from . import (default_scalar, engram_gate_bwd_fused, engram_gate_fwd, engram_gather_bwd,
+               engram_hash_gather)
 
 
 class EngramGateFunction(torch.autograd.Function):
@@ -50,9 +51,8 @@ class EngramGateFunction(torch.autograd.Function):
         if grad_out is None:
             grad_out = torch.zeros_like(x2)
         g = grad_out.reshape(-1, H).to(x2.dtype).contiguous()
-        dx, dk, dv, part = engram_gate_bwd(g, x2, k2, v2, wh.contiguous(), we.contiguous(),
-                                           ctx.eps, ctx.scalar)
-        dwh, dwe = engram_grad_w_reduce(part, wh.contiguous(), we.contiguous())
+        dx, dk, dv, dwh, dwe = engram_gate_bwd_fused(g, x2, k2, v2, wh.contiguous(),
+                                                     we.contiguous(), ctx.eps, ctx.scalar)
         lead = ctx.lead
         return (dx.view(*lead, H), dk.view(*lead, H), dv.view(*lead, H),
                 dwh.to(wh.dtype), dwe.to(we.dtype), None, None)

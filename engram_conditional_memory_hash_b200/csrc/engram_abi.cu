@@ -226,8 +226,32 @@ bool same_phase(std::initializer_list<const void *> ptrs)
     return true;
 }
 
-// CTAs of the generic gate kernels: up to 8 per SM, never more than tokens.
-int64_t generic_grid(const DeviceInfo &d, int64_t T) { return std::max<int64_t>(1, std::min<int64_t>(T, (int64_t)d.sms * 8)); }
+// CTAs of a generic gate kernel: as many as the SMs hold at once (one wave),
+// never more than tokens.
+template <typename K>
+engram_status_t generic_grid(const DeviceInfo &d, int64_t T, K kernel, size_t smem, int64_t *grid)
+{
+    int n = 0;
+    engram_status_t st = occupancy(kernel, engram::kGenThreads, smem, &n);
+    if (st != ENGRAM_OK) return st;
+    *grid = std::max<int64_t>(1, std::min<int64_t>(T, (int64_t)d.sms * std::max(n, 1)));
+    return ENGRAM_OK;
+}
+
+// Dynamic shared memory of the generic backward: its partial row, when it fits.
+size_t generic_bwd_smem(int H) { return H <= engram::kGenSmemPartial ? (size_t)H * 4 : 0; }
+
+// Partial rows (CTAs) of the generic backward: one wave of the kernel variant
+// with the fewer resident CTAs per SM.
+engram_status_t generic_bwd_grid(const DeviceInfo &d, int64_t T, int H, int64_t *grid)
+{
+    int64_t a = 0, b = 0;
+    const size_t smem = generic_bwd_smem(H);
+    engram_status_t st = generic_grid(d, T, engram::gate_generic_bwd_kernel<true>, smem, &a);
+    if (st == ENGRAM_OK) st = generic_grid(d, T, engram::gate_generic_bwd_kernel<false>, smem, &b);
+    *grid = std::min(a, b);
+    return st;
+}
 
 // -------------------------------------------------------------- launches ----
 
@@ -250,6 +274,35 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Launch of the tuned backward kernel; with tickets != NULL the kernel also
+// reduces the partial rows into dwh, dwe in its tail (engram_gate_bwd_fused).
+engram_status_t launch_gate_bwd_tuned(const DeviceInfo &dev, const void *grad_out, const void *x,
+                                      const void *k, const void *v, const void *wh, const void *we,
+                                      int64_t T, int32_t H, float eps, float scalar, void *dx, void *dk,
+                                      void *dv, float *w_partial, int64_t G, unsigned int *tickets,
+                                      float *dwh, float *dwe, cudaStream_t s)
+{
+    GateLaunch g;
+    engram_status_t st = gate_bwd_plan(dev, H, &g);
+    if (st != ENGRAM_OK) return st;
+    const engram::ReduceGroups grp = engram::reduce_groups(G);
+    auto args = [&](auto kern) -> engram_status_t {
+        kern<<<(unsigned)G, g.threads, g.smem, s>>>(
+            static_cast<const uint4 *>(grad_out), static_cast<const uint4 *>(x),
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<const uint4 *>(wh),
+            static_cast<const uint4 *>(we), T, H, eps, scalar, static_cast<uint4 *>(dx),
+            static_cast<uint4 *>(dk), static_cast<uint4 *>(dv), w_partial, g.nstage, tickets, grp, dwh,
+            dwe);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "gate_bwd launch");
+        return ENGRAM_OK;
+    };
+    if (g.maxv == 2 && g.threads <= kBwdNarrowThreads) return args(engram::gate_bwd_kernel<2, kBwdNarrowThreads>);
+    return g.maxv == 1 ? args(engram::gate_bwd_kernel<1>)
+         : g.maxv == 2 ? args(engram::gate_bwd_kernel<2>)
+                       : args(engram::gate_bwd_kernel<4>);
 }
 
 }  // namespace
@@ -379,7 +432,9 @@ engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, con
     if (!gate_tuned(H, {x, k, v, wh, we, out})) {
         auto kern = same_phase({x, k, v, out}) ? engram::gate_generic_fwd_kernel<true>
                                                : engram::gate_generic_fwd_kernel<false>;
-        kern<<<(unsigned)generic_grid(dev, T), engram::kGenThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        int64_t grid = 0;
+        if ((st = generic_grid(dev, T, kern, 0, &grid)) != ENGRAM_OK) return st;
+        kern<<<(unsigned)grid, engram::kGenThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
             static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(k),
             static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(wh),
             static_cast<const __nv_bfloat16 *>(we), T, H, eps, scalar, static_cast<__nv_bfloat16 *>(out),
@@ -416,7 +471,10 @@ int64_t engram_gate_bwd_num_partials(int64_t T, int32_t H)
     }
     DeviceInfo dev;
     if (device_info(&dev) != ENGRAM_OK) return -1;
-    if (!gate_tuned(H, {})) return generic_grid(dev, T);
+    if (!gate_tuned(H, {})) {
+        int64_t grid = 0;
+        return generic_bwd_grid(dev, T, H, &grid) == ENGRAM_OK ? grid : -1;
+    }
     GateLaunch g;
     if (gate_bwd_plan(dev, H, &g) != ENGRAM_OK) return -1;
     const int64_t full = (int64_t)dev.sms * g.ctas_per_sm;
@@ -448,7 +506,7 @@ engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void 
     if (!gate_tuned(H, {grad_out, x, k, v, wh, we, dx, dk, dv, w_partial})) {
         auto kern = same_phase({grad_out, x, k, v, dx, dk, dv}) ? engram::gate_generic_bwd_kernel<true>
                                                                  : engram::gate_generic_bwd_kernel<false>;
-        const size_t smem = H <= engram::kGenSmemPartial ? (size_t)H * 4 : 0;
+        const size_t smem = generic_bwd_smem(H);
         cudaError_t e0 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)(engram::kGenSmemPartial * 4));
         if (e0 != cudaSuccess) return cuda_fail(e0, "cudaFuncSetAttribute");
@@ -462,22 +520,8 @@ engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void 
         if (e != cudaSuccess) return cuda_fail(e, "gate_bwd launch");
         return ENGRAM_OK;
     }
-    GateLaunch g;
-    if ((st = gate_bwd_plan(dev, H, &g)) != ENGRAM_OK) return st;
-    auto args = [&](auto kern) -> engram_status_t {
-        kern<<<(unsigned)G, g.threads, g.smem, s>>>(
-            static_cast<const uint4 *>(grad_out), static_cast<const uint4 *>(x),
-            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<const uint4 *>(wh),
-            static_cast<const uint4 *>(we), T, H, eps, scalar, static_cast<uint4 *>(dx),
-            static_cast<uint4 *>(dk), static_cast<uint4 *>(dv), w_partial, g.nstage);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "gate_bwd launch");
-        return ENGRAM_OK;
-    };
-    if (g.maxv == 2 && g.threads <= kBwdNarrowThreads) return args(engram::gate_bwd_kernel<2, kBwdNarrowThreads>);
-    return g.maxv == 1 ? args(engram::gate_bwd_kernel<1>)
-         : g.maxv == 2 ? args(engram::gate_bwd_kernel<2>)
-                       : args(engram::gate_bwd_kernel<4>);
+    return launch_gate_bwd_tuned(dev, grad_out, x, k, v, wh, we, T, H, eps, scalar, dx, dk, dv, w_partial,
+                                 G, nullptr, nullptr, nullptr, s);
 }
 
 // ----------------------------------------------------------- grad_w_reduce ----
@@ -494,11 +538,44 @@ engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t G, int32_t 
     const unsigned blocks = (unsigned)((H + 31) / 32);
     // programmatic launch: scheduled while the backward kernel drains
     const cudaError_t e = launch_pdl(engram::grad_w_reduce_kernel, blocks, (unsigned)engram::kReduceThreads,
-                                     reinterpret_cast<cudaStream_t>(stream), w_partial, G, H,
+                                     reinterpret_cast<cudaStream_t>(stream), w_partial, G,
+                                     engram::reduce_groups(G), H,
                                      static_cast<const __nv_bfloat16 *>(wh),
                                      static_cast<const __nv_bfloat16 *>(we), dwh, dwe);
     if (e != cudaSuccess) return cuda_fail(e, "grad_w_reduce launch");
     return ENGRAM_OK;
+}
+
+// ---------------------------------------------------- gate bwd, fused reduce ----
+
+engram_status_t engram_gate_bwd_fused(const void *grad_out, const void *x, const void *k,
+                                      const void *v, const void *wh, const void *we, int64_t T,
+                                      int32_t H, float eps, float scalar, void *dx, void *dk, void *dv,
+                                      float *w_partial, int64_t G, uint32_t *tickets, float *dwh,
+                                      float *dwe, engram_stream_t stream)
+{
+    engram_status_t st = check_gate_common(T, H, eps, scalar);
+    if (st != ENGRAM_OK) return st;
+    if (!wh || !we || !w_partial || !tickets || !dwh || !dwe)
+        return fail(ENGRAM_ERR_INVALID_ARG, "wh, we, w_partial, tickets, dwh and dwe are required");
+    if (T > 0 && (!grad_out || !x || !k || !v || !dx || !dk || !dv))
+        return fail(ENGRAM_ERR_INVALID_ARG, "every tensor argument of engram_gate_bwd_fused is required");
+    if (G < 1 || G > 0x7fffffff) return fail(ENGRAM_ERR_INVALID_ARG, "G=%lld not in [1, 2^31-1]", (long long)G);
+    if (!aligned(grad_out, 2) || !aligned(x, 2) || !aligned(k, 2) || !aligned(v, 2) || !aligned(wh, 2) ||
+        !aligned(we, 2) || !aligned(dx, 2) || !aligned(dk, 2) || !aligned(dv, 2))
+        return fail(ENGRAM_ERR_INVALID_ARG, "bf16 tensors must be 2-byte aligned");
+    if (!aligned(w_partial, 4) || !aligned(tickets, 4) || !aligned(dwh, 4) || !aligned(dwe, 4))
+        return fail(ENGRAM_ERR_INVALID_ARG, "w_partial, tickets, dwh and dwe must be 4-byte aligned");
+    if (!gate_tuned(H, {grad_out, x, k, v, wh, we, dx, dk, dv, w_partial})) {
+        // generic shapes: the backward, then the standalone reduction (two launches)
+        st = engram_gate_bwd(grad_out, x, k, v, wh, we, T, H, eps, scalar, dx, dk, dv, w_partial, G, stream);
+        if (st != ENGRAM_OK) return st;
+        return engram_grad_w_reduce(w_partial, G, H, wh, we, dwh, dwe, stream);
+    }
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != ENGRAM_OK) return st;
+    return launch_gate_bwd_tuned(dev, grad_out, x, k, v, wh, we, T, H, eps, scalar, dx, dk, dv, w_partial, G,
+                                 tickets, dwh, dwe, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------ diagnostics ----
@@ -575,13 +652,16 @@ extern "C" engram_status_t engram_gate_bwd_noalloc(const void *grad_out, const v
     if (!dwh || !dwe) return fail(ENGRAM_ERR_INVALID_ARG, "dwh and dwe are required");
     if (!aligned(dwh, 4) || !aligned(dwe, 4))
         return fail(ENGRAM_ERR_INVALID_ARG, "dwh and dwe must be 4-byte aligned");
-    const int64_t G = engram_gate_bwd_num_partials(T, H);
+    int64_t G = engram_gate_bwd_num_partials(T, H);
     if (G < 1) return ENGRAM_ERR_CUDA;  // message set by engram_gate_bwd_num_partials
-    if ((size_t)G * (size_t)H > kNoAllocPartialFloats)
+    if ((size_t)H > kNoAllocPartialFloats)
         return fail(ENGRAM_ERR_UNSUPPORTED,
-                    "engram_gate_bwd_noalloc: %lld partial rows x H=%d need %lld floats of scratch, "
-                    "more than its static maximum of %zu",
-                    (long long)G, H, (long long)(G * H), kNoAllocPartialFloats);
+                    "engram_gate_bwd_noalloc: one partial row of H=%d floats exceeds its static scratch "
+                    "of %zu floats", H, kNoAllocPartialFloats);
+    // Fewer partial rows than recommended when they would not fit: the
+    // backward's CTAs loop over tokens, so any G >= 1 gives the same gradients
+    // (up to the order of the fp32 sums).
+    G = std::min<int64_t>(G, (int64_t)(kNoAllocPartialFloats / (size_t)H));
     float *scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != ENGRAM_OK) return st;
     // Every partial row the reduction reads is written by the backward first

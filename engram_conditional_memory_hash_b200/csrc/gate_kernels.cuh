@@ -278,6 +278,132 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
     }
 }
 
+// ------------------------------------------------ weight-gradient level 2 ----
+//
+// P_j = sum_p w_partial[p][j] over the G partial rows, in one order fixed by G
+// alone, so that the standalone reduction kernel and the tail fused into the
+// backward kernel give the same bits.  The rows form `count` consecutive
+// groups of `size` rows (the last one may be shorter):
+//     r_q = (((0 + Q_{q*size}) + Q_{q*size+1}) + ...)      in row order
+//     P   = (((0 + r_0) + r_1) + ...)                       in group order
+//     dwh_j = we_j * P_j,   dwe_j = wh_j * P_j
+// size = max(ceil(sqrt(G)), ceil(G / 32)), so that there are at most 32 groups
+// and, in the fused tail, the last CTA to finish reads about 2 sqrt(G) rows.
+
+struct ReduceGroups {
+    int64_t size;   // partial rows per group
+    int count;      // groups, 1..kMaxReduceGroups
+};
+
+constexpr int kMaxReduceGroups = 32;
+
+__host__ __device__ inline ReduceGroups reduce_groups(int64_t G)
+{
+    int64_t s = 1;
+    while (s * s < G) ++s;                   // ceil(sqrt(G)); G <= 2^31, a host-side call
+    const int64_t s32 = (G + kMaxReduceGroups - 1) / kMaxReduceGroups;
+    if (s32 > s) s = s32;
+    ReduceGroups g;
+    g.size = s;
+    g.count = (int)((G + s - 1) / s);
+    return g;
+}
+
+// Sum, for every float4 column f of the CTA's share (f = tid, tid + blockDim.x,
+// ...), the n rows base[(row0 + i * stride) * H ...], i = 0..n-1, in order
+// (starting from 0), then hand the sum to epi(f, sum).  Loads go through L2
+// only (the rows were written by other CTAs of the same grid) with 16 loads in
+// flight per thread.
+template <typename Epi>
+__device__ __forceinline__ void ordered_row_sum(const float *base, int64_t row0, int64_t n,
+                                                int64_t stride, int H, Epi epi)
+{
+    const int nf4 = H >> 2;
+    const int nt = blockDim.x;
+    for (int f0 = threadIdx.x; f0 < nf4; f0 += 4 * nt) {
+        float4 acc[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int64_t i = 0; i < n; i += 4) {
+            float4 v[4][4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float4 *row = reinterpret_cast<const float4 *>(base + (row0 + (i + r) * stride) * H);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (i + r < n && f0 + c * nt < nf4) v[r][c] = __ldcg(row + f0 + c * nt);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (i + r < n) {
+                        acc[c].x += v[r][c].x;
+                        acc[c].y += v[r][c].y;
+                        acc[c].z += v[r][c].z;
+                        acc[c].w += v[r][c].w;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (f0 + c * nt < nf4) epi(f0 + c * nt, acc[c]);
+    }
+}
+
+// dwh, dwe of the four columns 4f..4f+3 from their sums P.
+__device__ __forceinline__ void write_weight_grads(int f, float4 P, const __nv_bfloat16 *wh,
+                                                   const __nv_bfloat16 *we, float *dwh, float *dwe)
+{
+    const float p[4] = {P.x, P.y, P.z, P.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int j = 4 * f + e;
+        dwh[j] = __bfloat162float(we[j]) * p[e];
+        dwe[j] = __bfloat162float(wh[j]) * p[e];
+    }
+}
+
+// Level two fused into the tail of the backward kernel, with tickets instead
+// of a second launch and without any waiting: after writing its partial row a
+// CTA takes a ticket of its group; the CTA that takes the group's last ticket
+// sums the group's rows (in row order, into the group's first row) and takes
+// a ticket of the grid; the CTA that takes the grid's last ticket sums the
+// group rows (in group order), writes dwh and dwe, and sets every ticket back
+// to zero for the next call.  tickets[0] counts finished groups, tickets[1 + q]
+// the finished CTAs of group q.  `flag` is one word of shared memory.
+__device__ __noinline__ void grad_w_reduce_tail(float *w_partial, int64_t G, int H, ReduceGroups grp,
+                                                unsigned int *tickets, const __nv_bfloat16 *wh,
+                                                const __nv_bfloat16 *we, float *dwh, float *dwe,
+                                                unsigned int *flag)
+{
+    const int64_t q = (int64_t)blockIdx.x / grp.size;
+    const int64_t a = q * grp.size;
+    const int64_t n = (G - a < grp.size) ? G - a : grp.size;
+    __threadfence();              // this thread's partial-row stores, before the ticket
+    __syncthreads();
+    if (threadIdx.x == 0) *flag = atomicAdd(&tickets[1 + q], 1u) == (unsigned)(n - 1);
+    __syncthreads();
+    if (*flag == 0) return;
+    __threadfence();              // the group's rows, after its last ticket
+
+    ordered_row_sum(w_partial, a, n, 1, H, [&](int f, float4 r) {
+        reinterpret_cast<float4 *>(w_partial + a * H)[f] = r;
+    });
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) *flag = atomicAdd(&tickets[0], 1u) == (unsigned)(grp.count - 1);
+    __syncthreads();
+    if (*flag == 0) return;
+    __threadfence();
+
+    ordered_row_sum(w_partial, 0, grp.count, grp.size, H,
+                    [&](int f, float4 P) { write_weight_grads(f, P, wh, we, dwh, dwe); });
+    // every other CTA has taken all of its tickets: reset them for the next call
+    for (int i = threadIdx.x; i <= grp.count; i += blockDim.x) tickets[i] = 0u;
+}
+
 // -------------------------------------------------------------- backward ----
 
 // Backward kernel with MAXV vectors per thread and at most MAXT threads per
@@ -291,7 +417,8 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
                 const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                 const uint4 *__restrict__ wh, const uint4 *__restrict__ we, int64_t T, int H,
                 float eps, float scalar, uint4 *__restrict__ dx, uint4 *__restrict__ dk,
-                uint4 *__restrict__ dv, float *__restrict__ w_partial, int nstage)
+                uint4 *__restrict__ dv, float *w_partial, int nstage,
+                unsigned int *tickets, ReduceGroups grp, float *dwh, float *dwe)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     const int nvec = H >> 3;
@@ -385,11 +512,13 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
             rbd[warp] = pa;
         }
         if (__syncthreads_or(!ok)) {
+            // Give up on the remaining tokens but still take part in the
+            // weight-gradient tail below, so that its tickets stay consistent.
             if (tid == 0) {
                 record_device_error(kErrPipelineTimeout);
                 gate_drain(bar0, i, nrows, nstage);
             }
-            return;
+            break;
         }
         if (tid == 0 && i + nstage < nrows)
             gate_issue_row<4>(smem, bar0, src, first + (i + nstage) * G, row_bytes, s);
@@ -449,19 +578,23 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
             prow[2 * vi + 1] = make_float4(acc[m][2].x, acc[m][2].y, acc[m][3].x, acc[m][3].y);
         }
     }
+    if (tickets != nullptr)
+        grad_w_reduce_tail(w_partial, G, H, grp, tickets, reinterpret_cast<const __nv_bfloat16 *>(wh),
+                           reinterpret_cast<const __nv_bfloat16 *>(we), dwh, dwe,
+                           reinterpret_cast<unsigned int *>(red));
 }
 
-// ------------------------------------------------ weight-gradient level 2 ----
+// ------------------------------------------ standalone weight-gradient level 2 ----
 
 constexpr int kReduceThreads = 1024;
 constexpr int kReduceWarps = kReduceThreads / 32;
+static_assert(kReduceWarps >= kMaxReduceGroups, "one warp per group");
 
-// P_j = sum_{p<G} w_partial[p][j] for the 32 columns of a block: warp q sums
-// partial rows p = q, q + 32, q + 64, ... in order, then warp 0 adds the 32
-// warp sums in warp order, so the result depends only on G.  dwh = we * P,
-// dwe = wh * P.
+// Standalone level two, in the order above: per block of 32 columns, warp q
+// sums the rows of group q in order, then warp 0 adds the group sums in group
+// order.
 __global__ void __launch_bounds__(kReduceThreads)
-grad_w_reduce_kernel(const float *__restrict__ w_partial, int64_t G, int H,
+grad_w_reduce_kernel(const float *__restrict__ w_partial, int64_t G, ReduceGroups grp, int H,
                      const __nv_bfloat16 *__restrict__ wh, const __nv_bfloat16 *__restrict__ we,
                      float *__restrict__ dwh, float *__restrict__ dwe)
 {
@@ -472,25 +605,25 @@ grad_w_reduce_kernel(const float *__restrict__ w_partial, int64_t G, int H,
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int col = blockIdx.x * 32 + lane;
     float a = 0.f;
-    if (col < H) {
+    if (col < H && warp < grp.count) {
         const float *p = w_partial + col;
-        int64_t q = warp;
-        for (; q + 3 * kReduceWarps < G; q += 4 * kReduceWarps) {
-            const float v0 = p[q * H], v1 = p[(q + kReduceWarps) * H],
-                        v2 = p[(q + 2 * kReduceWarps) * H], v3 = p[(q + 3 * kReduceWarps) * H];
+        const int64_t p0 = (int64_t)warp * grp.size;
+        const int64_t p1 = (G - p0 < grp.size) ? G : p0 + grp.size;
+        int64_t r = p0;
+        for (; r + 3 < p1; r += 4) {
+            const float v0 = p[r * H], v1 = p[(r + 1) * H], v2 = p[(r + 2) * H], v3 = p[(r + 3) * H];
             a += v0;
             a += v1;
             a += v2;
             a += v3;
         }
-        for (; q < G; q += kReduceWarps) a += p[q * H];
+        for (; r < p1; ++r) a += p[r * H];
     }
     part[warp][lane] = a;
     __syncthreads();
     if (warp == 0 && col < H) {
         float P = 0.f;
-#pragma unroll
-        for (int q = 0; q < kReduceWarps; ++q) P += part[q][lane];
+        for (int q = 0; q < grp.count; ++q) P += part[q][lane];
         dwh[col] = __bfloat162float(we[col]) * P;
         dwe[col] = __bfloat162float(wh[col]) * P;
     }

@@ -17,9 +17,14 @@
 //      sets the row's bit in `dupmap` (which entry arrives first does not
 //      matter: a row ends up in dupmap exactly when two or more entries read it);
 //   2. unique: entries whose row is not in dupmap update their row directly
-//      with one rounding: fp32((double)d_tables[r] + g); each tile stages the
-//      (key, e) pairs of its other entries in position order, with their
-//      count and first-digit histogram;
+//      with one rounding: fp32((double)d_tables[r] + g).  This is the
+//      bandwidth-bound part; it runs on a persistent grid that leaves room on
+//      every SM, and the list kernels below (stage, sort, segments) are
+//      scheduled beside it at once (they touch only rows in dupmap, it only
+//      the others);
+//      stage: each tile of entries stages the (key, e) pairs of its entries
+//      whose row is in dupmap, in position order, with their count and
+//      first-digit histogram;
 //   3. a stable least-significant-digit radix sort of the staged entries by
 //      key, 8 bits per pass: a per-tile digit histogram, an exclusive scan of
 //      each digit's counts over the tiles, and a scatter whose within-tile
@@ -56,7 +61,7 @@ constexpr int kSortWarps = kSortThreads / 32;
 constexpr int kSortRounds = 4;
 constexpr int kSortTile = kSortThreads * kSortRounds;   // list entries per CTA tile
 constexpr int kRadixBins = 256;
-constexpr int kScanThreads = 1024;
+constexpr int kScanThreads = 256;
 constexpr int kSegChunk = 64;                           // sorted entries per warp
 constexpr int kSegThreads = 256;
 constexpr int kCarryThreads = 256;
@@ -103,6 +108,13 @@ __device__ __forceinline__ bool row_bit(const uint32_t *__restrict__ map, uint32
     return (map[key >> 5] >> (key & 31u)) & 1u;
 }
 
+// The same, read through L2 only (for a kernel that does not wait for its
+// predecessor: the bitmap was written two kernels earlier).
+__device__ __forceinline__ bool row_bit_l2(const uint32_t *__restrict__ map, uint32_t key)
+{
+    return (__ldcg(map + (key >> 5)) >> (key & 31u)) & 1u;
+}
+
 // ------------------------------------------------------- mark and unique ----
 
 // seen/dupmap bits of every entry's row (both bitmaps zeroed before the
@@ -134,36 +146,93 @@ gbwd_mark_kernel(const int64_t *__restrict__ idx, const __grid_constant__ Gather
 }
 
 // Rows read by one entry only: d_tables[r] = fp32((double)d_tables[r] + g).
-// The entries of the other rows are staged for the sort, in position order:
-// tile t (entries [t * kUniqTile, (t + 1) * kUniqTile)) writes the (key, e)
-// pairs of its listed entries to stage_keys/stage_vals[t * kUniqTile ...],
-// their count to tile_cnt[t], the histogram of their lowest 8 key bits to
-// hist[digit * ntiles + t] (the first radix pass reads the staged tiles
-// directly), and adds the count to *m_out, the length of the list.
-// Warp w of the CTA handles kUniqWarpEntries entries in rounds of 32 (lane l:
-// the round's entry l); a round's unique entries are dealt to the warp's
-// 32 / LPR groups of LPR lanes, U at a time per group, lane cv owning the
-// columns [8 cv, 8 cv + 8).
-// Four CTAs per SM (64 registers a thread): more resident warps outweigh the
-// few registers spilled (218 -> 209 us per call at the full-path workload).
+// Persistent: CTA b handles the tiles b, b + gridDim.x, ... of kUniqTile
+// entries; warp w of a tile handles kUniqWarpEntries entries in rounds of 32
+// (lane l: the round's entry l); a round's unique entries are dealt to the
+// warp's 32 / LPR groups of LPR lanes, U at a time per group, lane cv owning
+// the columns [8 cv, 8 cv + 8).  The kernel releases its dependents as soon
+// as it starts, and its grid leaves one CTA slot per SM free, so that the
+// staging and list kernels launched after it run beside it.  Up to four CTAs
+// per SM fit (64 registers a thread, a few spilled).
 template <int LPR, int U>
 __global__ void __launch_bounds__(kUniqThreads, 4)
 gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_rows,
                    const __grid_constant__ GatherBwdParams p, const uint32_t *__restrict__ dupmap,
-                   float4 *__restrict__ d_tables, uint32_t *__restrict__ stage_keys,
-                   uint32_t *__restrict__ stage_vals, uint32_t *__restrict__ tile_cnt,
-                   uint32_t *__restrict__ hist, uint32_t *__restrict__ m_out)
+                   float4 *__restrict__ d_tables)
 {
     constexpr int GPW = 32 / LPR;
     constexpr int RW = kUniqWarpEntries / 32;
-    __shared__ uint32_t warp_cnt[kUniqThreads / 32];
-    __shared__ uint32_t sh[kRadixBins];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int grp = lane / LPR, cv = lane % LPR;
     const int nv = p.D >> 3;
     const bool col = cv < nv;
-    sh[threadIdx.x] = 0u;
     pdl_wait_and_release();
+    const int64_t ntiles = (p.N + kUniqTile - 1) / kUniqTile;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t base = tile * kUniqTile + (int64_t)warp * kUniqWarpEntries;
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int64_t e = base + r * 32 + lane;
+            const uint32_t key = e < p.N ? gbwd_key(idx, e, p, false) : p.R;
+            const bool uniq = key < p.R && !row_bit(dupmap, key);
+            const uint32_t um = __ballot_sync(0xffffffffu, uniq);
+            if (um == 0u) continue;
+            for (int j0 = 0; j0 < 32; j0 += GPW * U) {
+                uint4 g[U];
+                float4 o0[U], o1[U];
+                uint32_t k[U];
+                bool on[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int j = j0 + u * GPW + grp;
+                    k[u] = __shfl_sync(0xffffffffu, key, j);
+                    on[u] = ((um >> j) & 1u) && col;
+                    if (on[u]) {
+                        g[u] = __ldg(d_rows + (base + r * 32 + j) * nv + cv);
+                        const float4 *t = d_tables + (int64_t)k[u] * (2 * nv) + 2 * cv;
+                        o0[u] = t[0];
+                        o1[u] = t[1];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (!on[u]) continue;
+                    float4 *t = d_tables + (int64_t)k[u] * (2 * nv) + 2 * cv;
+                    t[0] = make_float4((float)((double)o0[u].x + (double)bf16_lo(g[u].x)),
+                                       (float)((double)o0[u].y + (double)bf16_hi(g[u].x)),
+                                       (float)((double)o0[u].z + (double)bf16_lo(g[u].y)),
+                                       (float)((double)o0[u].w + (double)bf16_hi(g[u].y)));
+                    t[1] = make_float4((float)((double)o1[u].x + (double)bf16_lo(g[u].z)),
+                                       (float)((double)o1[u].y + (double)bf16_hi(g[u].z)),
+                                       (float)((double)o1[u].z + (double)bf16_lo(g[u].w)),
+                                       (float)((double)o1[u].w + (double)bf16_hi(g[u].w)));
+                }
+            }
+        }
+    }
+}
+
+// The entries of rows in dupmap, staged for the sort in position order: tile t
+// (entries [t * kUniqTile, (t + 1) * kUniqTile)) writes their (key, e) pairs to
+// stage_keys/stage_vals[t * kUniqTile ...], their count to tile_cnt[t], the
+// histogram of their lowest 8 key bits to hist[digit * ntiles + t] (the first
+// radix pass reads the staged tiles directly), and adds the count to *m_out,
+// the length of the list.
+// Launched right after the unique-row update and run beside it: it does not
+// wait for that kernel (which it does not depend on) and reads dupmap, which
+// the mark kernel wrote before the update kernel started, through L2.
+__global__ void __launch_bounds__(kUniqThreads)
+gbwd_stage_kernel(const int64_t *__restrict__ idx, const __grid_constant__ GatherBwdParams p,
+                  const uint32_t *__restrict__ dupmap, uint32_t *__restrict__ stage_keys,
+                  uint32_t *__restrict__ stage_vals, uint32_t *__restrict__ tile_cnt,
+                  uint32_t *__restrict__ hist, uint32_t *__restrict__ m_out)
+{
+    constexpr int RW = kUniqWarpEntries / 32;
+    __shared__ uint32_t warp_cnt[kUniqThreads / 32];
+    __shared__ uint32_t sh[kRadixBins];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    sh[threadIdx.x] = 0u;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t base = (int64_t)blockIdx.x * kUniqTile + (int64_t)warp * kUniqWarpEntries;
     uint32_t key[RW], dmask[RW];
     uint32_t ndup = 0;
@@ -171,45 +240,9 @@ gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_
     for (int r = 0; r < RW; ++r) {
         const int64_t e = base + r * 32 + lane;
         key[r] = e < p.N ? gbwd_key(idx, e, p, false) : p.R;
-        const bool dup = key[r] < p.R && row_bit(dupmap, key[r]);
-        dmask[r] = __ballot_sync(0xffffffffu, dup);
+        dmask[r] = __ballot_sync(0xffffffffu, key[r] < p.R && row_bit_l2(dupmap, key[r]));
         ndup += (uint32_t)__popc(dmask[r]);
-        const uint32_t um = __ballot_sync(0xffffffffu, key[r] < p.R && !dup);
-        if (um == 0u) continue;
-        for (int j0 = 0; j0 < 32; j0 += GPW * U) {
-            uint4 g[U];
-            float4 o0[U], o1[U];
-            uint32_t k[U];
-            bool on[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int j = j0 + u * GPW + grp;
-                k[u] = __shfl_sync(0xffffffffu, key[r], j);
-                on[u] = ((um >> j) & 1u) && col;
-                if (on[u]) {
-                    g[u] = __ldg(d_rows + (base + r * 32 + j) * nv + cv);
-                    const float4 *t = d_tables + (int64_t)k[u] * (2 * nv) + 2 * cv;
-                    o0[u] = t[0];
-                    o1[u] = t[1];
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                if (!on[u]) continue;
-                float4 *t = d_tables + (int64_t)k[u] * (2 * nv) + 2 * cv;
-                t[0] = make_float4((float)((double)o0[u].x + (double)bf16_lo(g[u].x)),
-                                   (float)((double)o0[u].y + (double)bf16_hi(g[u].x)),
-                                   (float)((double)o0[u].z + (double)bf16_lo(g[u].y)),
-                                   (float)((double)o0[u].w + (double)bf16_hi(g[u].y)));
-                t[1] = make_float4((float)((double)o1[u].x + (double)bf16_lo(g[u].z)),
-                                   (float)((double)o1[u].y + (double)bf16_hi(g[u].z)),
-                                   (float)((double)o1[u].z + (double)bf16_lo(g[u].w)),
-                                   (float)((double)o1[u].w + (double)bf16_hi(g[u].w)));
-            }
-        }
     }
-
-    // stage the listed entries of this tile in position order
     if (lane == 0) warp_cnt[warp] = ndup;
     __syncthreads();
     uint32_t off = 0, tot = 0;

@@ -7,6 +7,13 @@ namespace {
 
 constexpr int64_t kGbwdMaxEntries = int64_t(1) << 30;
 
+// CTAs per SM of the persistent unique-row update (it could hold four; the
+// fourth slot is left to the staging and list kernels that run beside it).
+#ifndef ENGRAM_GBWD_UNIQ_PER_SM
+#define ENGRAM_GBWD_UNIQ_PER_SM 3
+#endif
+constexpr int kGbwdUniqPerSm = ENGRAM_GBWD_UNIQ_PER_SM;
+
 // Offsets (bytes, 256-aligned) of the gather backward's scratch in the
 // caller's workspace.  A region zeroed by every call first: the `seen` and
 // `dupmap` bitmaps (one bit per table row) and the counters (list length,
@@ -119,6 +126,8 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     if (workspace_bytes < g.total)
         return fail(ENGRAM_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, g.total);
 
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != ENGRAM_OK) return st;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     uint32_t *seen = reinterpret_cast<uint32_t *>(ws + g.seen);
     uint32_t *dupmap = reinterpret_cast<uint32_t *>(ws + g.dupmap);
@@ -146,25 +155,27 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
         e = launch_pdl(engram::gbwd_mark_kernel, mblocks, (unsigned)engram::kMarkThreads, s, idx, p, seen,
                        dupmap);
     }
-    // 2. rows read once: update in place; stage the rest per tile (into the
-    //    second buffer pair), with the first radix pass's tile histograms
+    // 2. rows read once: update in place, on a persistent grid that leaves a
+    //    CTA slot free on every SM; the kernels from 3 on run beside it
     if (e == cudaSuccess) {
-        const unsigned ub = (unsigned)g.utiles, ut = (unsigned)engram::kUniqThreads;
+        const unsigned ub = (unsigned)std::min<int64_t>(g.utiles, (int64_t)dev.sms * kGbwdUniqPerSm);
+        const unsigned ut = (unsigned)engram::kUniqThreads;
         const uint32_t *dm = dupmap;
         if (nv <= 4)
-            e = launch_pdl(engram::gbwd_unique_kernel<4, 4>, ub, ut, s, idx, rows, p, dm, tab4, keys[1], vals[1],
-                           tile_cnt, hist, m_dev);
+            e = launch_pdl(engram::gbwd_unique_kernel<4, 4>, ub, ut, s, idx, rows, p, dm, tab4);
         else if (nv <= 8)
-            e = launch_pdl(engram::gbwd_unique_kernel<8, 4>, ub, ut, s, idx, rows, p, dm, tab4, keys[1], vals[1],
-                           tile_cnt, hist, m_dev);
+            e = launch_pdl(engram::gbwd_unique_kernel<8, 4>, ub, ut, s, idx, rows, p, dm, tab4);
         else if (nv <= 16)
-            e = launch_pdl(engram::gbwd_unique_kernel<16, 4>, ub, ut, s, idx, rows, p, dm, tab4, keys[1],
-                           vals[1], tile_cnt, hist, m_dev);
+            e = launch_pdl(engram::gbwd_unique_kernel<16, 4>, ub, ut, s, idx, rows, p, dm, tab4);
         else
-            e = launch_pdl(engram::gbwd_unique_kernel<32, 4>, ub, ut, s, idx, rows, p, dm, tab4, keys[1],
-                           vals[1], tile_cnt, hist, m_dev);
+            e = launch_pdl(engram::gbwd_unique_kernel<32, 4>, ub, ut, s, idx, rows, p, dm, tab4);
     }
-    // 3. stable radix sort by row of the staged entries into a contiguous
+    // 3. the entries of rows read more than once, staged per tile (into the
+    //    second buffer pair) with the first radix pass's tile histograms
+    if (e == cudaSuccess)
+        e = launch_pdl(engram::gbwd_stage_kernel, (unsigned)g.utiles, (unsigned)engram::kUniqThreads, s, idx,
+                       p, static_cast<const uint32_t *>(dupmap), keys[1], vals[1], tile_cnt, hist, m_dev);
+    // 4. stable radix sort by row of the staged entries into a contiguous
     //    list; keys lie in [0, R): sort on the bit length of R - 1
     int nbits = 0;
     while (nbits < 32 && (uint64_t(R - 1) >> nbits) != 0) ++nbits;
@@ -189,7 +200,7 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
                            keys[1 - cur], vals[1 - cur]);
         cur = 1 - cur;
     }
-    // 4. segments of the sorted list, then the segments that cross chunks
+    // 5. segments of the sorted list, then the segments that cross chunks
     const int64_t seg_blocks = (g.nchunks + engram::kSegThreads / 32 - 1) / (engram::kSegThreads / 32);
     const unsigned blocks = (unsigned)std::min<int64_t>(seg_blocks, int64_t(1) << 30);
     const unsigned S_ = engram::kSegThreads;
@@ -208,7 +219,10 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
             e = launch_pdl(engram::gbwd_segment_kernel<32, 2>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
     }
-    // one warp per listed chunk (a warp loops when more than 4096 are listed)
+    // one warp per listed chunk (a warp loops when more than 4096 are listed);
+    // launched without the programmatic dependency, so that it starts only
+    // when everything before it in the stream (the unique-row update included)
+    // has completed, and the call's last kernel ends after all of its work
     const int64_t carry_warps = std::min<int64_t>(g.nchunks, 4096);
     const unsigned carry_blocks = (unsigned)((carry_warps + engram::kCarryThreads / 32 - 1) /
                                              (engram::kCarryThreads / 32));
@@ -216,14 +230,14 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     const double *ca = carry_a, *cb = carry_b;
     const uint32_t *cl = carry_list, *cn = carry_count;
     if (e == cudaSuccess) {
-        if (D <= 32)
-            e = launch_pdl(engram::gbwd_carry_kernel<1>, carry_blocks, CT, s, kc, p, d_tables, ca, cb, cl, cn);
-        else if (D <= 64)
-            e = launch_pdl(engram::gbwd_carry_kernel<2>, carry_blocks, CT, s, kc, p, d_tables, ca, cb, cl, cn);
-        else if (D <= 128)
-            e = launch_pdl(engram::gbwd_carry_kernel<4>, carry_blocks, CT, s, kc, p, d_tables, ca, cb, cl, cn);
-        else
-            e = launch_pdl(engram::gbwd_carry_kernel<8>, carry_blocks, CT, s, kc, p, d_tables, ca, cb, cl, cn);
+        auto carry = [&](auto kern) {
+            kern<<<carry_blocks, CT, 0, s>>>(kc, p, d_tables, ca, cb, cl, cn);
+            return cudaGetLastError();
+        };
+        e = D <= 32 ? carry(engram::gbwd_carry_kernel<1>)
+          : D <= 64 ? carry(engram::gbwd_carry_kernel<2>)
+          : D <= 128 ? carry(engram::gbwd_carry_kernel<4>)
+                     : carry(engram::gbwd_carry_kernel<8>);
     }
     if (e != cudaSuccess) return cuda_fail(e, "gather_bwd launch");
     return ENGRAM_OK;

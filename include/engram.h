@@ -227,10 +227,15 @@ ENGRAM_API engram_status_t engram_gate_bwd(const void *grad_out, const void *x, 
 
 /*
  * engram_grad_w_reduce - weight-gradient reduction ("engram_grad_w_reduce"):
- *     P_j   = sum_{p=0}^{G-1} w_partial[p][j]   (fixed order, deterministic)
+ *     P_j   = sum_{p=0}^{G-1} w_partial[p][j]
  *     dwh_j = we_j * P_j,   dwe_j = wh_j * P_j
  * which are the gradients of sum over tokens of the forward's loss with
- * respect to wh and we.
+ * respect to wh and we.  The fp32 sum has an order fixed by G alone, so the
+ * result is bitwise reproducible: the rows form consecutive groups of
+ * size = max(ceil(sqrt(G)), ceil(G/32)) rows (the last group may be shorter),
+ * each group is summed in row order starting from 0, and the group sums are
+ * added in group order starting from 0.  engram_gate_bwd_fused uses the same
+ * order, so both give the same bits.
  *
  * w_partial   device, fp32 [G*H] as written by engram_gate_bwd, 4-byte aligned.
  * G >= 1, H >= 1.
@@ -240,6 +245,43 @@ ENGRAM_API engram_status_t engram_gate_bwd(const void *grad_out, const void *x, 
 ENGRAM_API engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t G, int32_t H,
                                      const void *wh, const void *we, float *dwh, float *dwe,
                                      engram_stream_t stream);
+
+/* Words of the ticket array engram_gate_bwd_fused takes. */
+#define ENGRAM_GATE_BWD_TICKETS 64
+
+/*
+ * engram_gate_bwd_fused - engram_gate_bwd and engram_grad_w_reduce in one
+ * launch (the page lists the two operators separately; here the reduction of
+ * the partial rows runs in the tail of the backward kernel instead of a
+ * second kernel).  Each CTA of the backward writes its partial row and takes
+ * a ticket (an atomic count) of its group of rows; the CTA that completes a
+ * group sums that group's rows, and the CTA that completes the last group
+ * sums the group sums and writes dwh and dwe.  No CTA waits for another.
+ * The order of every fp32 sum is the one engram_grad_w_reduce documents, so
+ * dwh and dwe are bitwise those of engram_gate_bwd followed by
+ * engram_grad_w_reduce with the same G.
+ *
+ * Arguments as in engram_gate_bwd, plus:
+ * w_partial   device, fp32 [G*H], 4-byte aligned: scratch of the reduction
+ *             (its contents on return are unspecified: group rows hold sums).
+ * tickets     device, uint32 [ENGRAM_GATE_BWD_TICKETS], 4-byte aligned, all
+ *             zero before the first call (e.g. cudaMemsetAsync once).  Every
+ *             call sets them back to zero when it completes, so one array
+ *             serves any number of calls in stream order; calls that may run
+ *             at the same time on the GPU need separate arrays.  After a call
+ *             that recorded ENGRAM_DEVICE_ERR_PIPELINE_TIMEOUT its gradients are
+ *             invalid (the tickets are still reset).
+ * dwh, dwe    device, fp32 [H], 4-byte aligned; overwritten, not accumulated.
+ * Shapes that the tuned kernels do not take (see the conventions) run the
+ * generic backward and then the standalone reduction: two launches, same
+ * results as those two calls, tickets untouched.
+ */
+ENGRAM_API engram_status_t engram_gate_bwd_fused(const void *grad_out, const void *x,
+                                      const void *k, const void *v, const void *wh,
+                                      const void *we, int64_t T, int32_t H, float eps,
+                                      float scalar, void *dx, void *dk, void *dv,
+                                      float *w_partial, int64_t G, uint32_t *tickets,
+                                      float *dwh, float *dwe, engram_stream_t stream);
 
 /*
  * engram_gate_bwd_noalloc - engram_gate_bwd followed by engram_grad_w_reduce,
@@ -253,9 +295,13 @@ ENGRAM_API engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t 
  * rows are kept in a static device array of the library (8 MiB per GPU that
  * loads it, held until the process exits) instead of a caller buffer, and the
  * reduced gradients dwh, dwe (device, fp32 [H], 4-byte aligned, overwritten)
- * are written directly.  The partial row count is the one
- * engram_gate_bwd_num_partials(T, H) recommends; if those rows need more than
- * 2^21 floats the call returns ENGRAM_ERR_UNSUPPORTED and launches nothing.
+ * are written directly.  The partial row count G is the one
+ * engram_gate_bwd_num_partials(T, H) recommends, lowered to floor(2^21 / H)
+ * when G rows of H floats would not fit in the array (the backward's CTAs
+ * loop over tokens, so any G gives the same gradients up to the order of the
+ * fp32 sums).  H itself is limited to 65536 as everywhere, so one row always
+ * fits; sizes outside the gate's limits return ENGRAM_ERR_UNSUPPORTED or
+ * ENGRAM_ERR_INVALID_ARG and launch nothing.
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current): make that first call before any stream

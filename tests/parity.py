@@ -63,3 +63,34 @@ def assert_dw_close(name, got: torch.Tensor, want: np.ndarray):
 
 def ill_conditioned(s_ref: np.ndarray) -> np.ndarray:
     return np.abs(s_ref) < ILL_S
+
+
+def check_gate_blockwise(o, gi, res, eps, blk=2048, forward=True):
+    """Compare every element of the GPU's per-token gate outputs (out, gate,
+    dx, dk, dv in `res`, torch tensors [T, H] / [T]) with the oracle, computed
+    block by block of `blk` tokens so that the fp64 arrays stay small.
+    Returns the oracle's dwh, dwe summed over the blocks (the weight gradient
+    is linear in the tokens) and s for every token."""
+    T, H = gi["x"].shape
+    dw = {"dwh": np.zeros(H), "dwe": np.zeros(H)}
+    s_all = np.empty(T)
+    for a in range(0, T, blk):
+        sl = slice(a, min(T, a + blk))
+        sub = {n: (arr[sl] if arr.ndim == 2 else arr) for n, arr in gi.items()}
+        if forward:
+            ref_out, ref_gate = o.engram_gate_fwd(sub["x"], sub["k"], sub["v"], sub["wh"],
+                                                  sub["we"], eps=eps)
+            assert_bf16_close("out", res["out"][sl], ref_out)
+            assert_gate_close(res["gate"][sl], ref_gate)
+            del ref_out
+        ref = o.engram_gate_bwd(sub["g"], sub["x"], sub["k"], sub["v"], sub["wh"], sub["we"],
+                                eps=eps)
+        ill = ill_conditioned(ref["s"])
+        assert_bf16_close("dx", res["dx"][sl], ref["dx"], rows_relaxed=ill)
+        assert_bf16_close("dk", res["dk"][sl], ref["dk"], rows_relaxed=ill)
+        assert_bf16_close("dv", res["dv"][sl], ref["dv"])
+        dw["dwh"] += ref["dwh"]
+        dw["dwe"] += ref["dwe"]
+        s_all[sl] = ref["s"]
+        del ref
+    return dw, s_all

@@ -78,6 +78,42 @@ def test_gate_bwd_rejects_before_launch():
     assert bwd(part=ctypes.c_void_p(18)) == INVALID                 # fp32 partials not 4-aligned
 
 
+def test_gate_bwd_fused_rejects_before_launch():
+    L = eng.lib()
+    p = ctypes.c_void_p(16)
+
+    def fused(G=1, H=64, ptr=p, part=p, tickets=p, dwh=p, dwe=p, T=4):
+        return L.engram_gate_bwd_fused(p, p, p, p, p, p, T, H, 1e-6, 0.125, ptr, p, p, part, G,
+                                       tickets, dwh, dwe, None)
+
+    assert fused(G=0) == INVALID
+    assert fused(G=2**31) == INVALID
+    assert fused(H=0) == UNSUPPORTED and fused(H=70000) == UNSUPPORTED
+    assert fused(ptr=None) == INVALID
+    assert fused(tickets=None) == INVALID
+    assert b"tickets" in L.engram_last_error()
+    assert fused(dwh=None) == INVALID and fused(dwe=None) == INVALID
+    assert fused(tickets=ctypes.c_void_p(18)) == INVALID             # tickets not 4-aligned
+    assert fused(dwe=ctypes.c_void_p(18)) == INVALID
+    assert fused(part=ctypes.c_void_p(18)) == INVALID
+    assert fused(T=-1) == INVALID
+
+
+def test_gate_bwd_noalloc_rejects_before_launch():
+    L = eng.lib()
+    p = ctypes.c_void_p(16)
+
+    def noalloc(H=64, T=4, dwh=p):
+        return L.engram_gate_bwd_noalloc(p, p, p, p, p, p, T, H, 1e-6, 0.125, p, p, p, dwh, p,
+                                         None)
+
+    # H beyond the gate's limit is refused before any device query or launch
+    assert noalloc(H=65544) == UNSUPPORTED
+    assert noalloc(H=0) == UNSUPPORTED
+    assert noalloc(T=-1) == INVALID
+    assert noalloc(dwh=None) == INVALID
+
+
 def test_grad_w_reduce_rejects_before_launch():
     L = eng.lib()
     p = ctypes.c_void_p(16)

@@ -14,9 +14,18 @@ def test_algorithmic_bytes_full_path():
     assert ab["hash_gather"] == T * (8 + 16 * 8 + 2 * 16 * 128) == 277348352
     # gate forward: x, k, v read, out written (2H bytes each), gate written, wh, we read
     assert ab["gate_fwd"] == T * (8 * H + 4) + 4 * H
-    # gate backward: g, x, k, v read, dx, dk, dv written, partial rows, wh, we
-    assert ab["gate_bwd"] == T * 14 * H + G * 4 * H + 4 * H
-    assert ab["grad_w_reduce"] == G * 4 * H + 8 * H + 4 * H
+    # fused gate backward: g, x, k, v read, dx, dk, dv written, partial rows
+    # written, wh, we read; then the reduction: partial rows read, dwh, dwe
+    # written, wh, we read
+    assert ab["gate_bwd"] == (T * 14 * H + G * 4 * H + 4 * H) + (G * 4 * H + 8 * H + 4 * H)
+    assert set(ab) == {"hash_gather", "gate_fwd", "gate_bwd"}
+
+
+def test_kernel_entry_fractions():
+    e = bench.kernel_entry(100.0, 560_000_000, 7000.0)        # 5.6 TB/s
+    assert e["GB/s"] == 5600.0
+    assert e["frac"] == 0.8 and e["frac_nominal"] == 0.7
+    assert e["us_at_bar"] == 100.0                            # exactly at 70% of 8 TB/s
 
 
 def test_gather_bwd_bytes():
@@ -30,7 +39,7 @@ def test_gather_bwd_bytes():
 
 
 def test_every_kernel_has_sources_and_a_digest():
-    for k in ("hash_gather", "gate_fwd", "gate_bwd", "grad_w_reduce", "gather_bwd"):
+    for k in ("hash_gather", "gate_fwd", "gate_bwd", "gather_bwd"):
         d = bench.source_digest(k)
         assert len(d) == 16 and int(d, 16) >= 0
     # the gate kernels share their sources, the gather backward has its own

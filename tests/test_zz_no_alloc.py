@@ -41,7 +41,9 @@ def _allocating(t):
     return dx, dk, dv, dwh, dwe
 
 
-@pytest.mark.parametrize("T,H", [(2048, 7168), (333, 4096)])
+# (1500, 2049) and (300, 16384) run the generic kernels, whose recommended
+# partial-row count would not fit in the static scratch: the call lowers it
+@pytest.mark.parametrize("T,H", [(2048, 7168), (333, 4096), (1500, 2049), (300, 16384)])
 def test_noalloc_matches_allocating_entry_points(T, H):
     for call, index in enumerate((200, 201)):          # two calls in a row
         t = _inputs(index + H % 7, T, H)
@@ -55,6 +57,19 @@ def test_noalloc_matches_allocating_entry_points(T, H):
         for name, a, b in zip(("dwh", "dwe"), got[3:], want[3:]):
             ga, wb = f64(a), f64(b)
             assert np.abs(ga - wb).max() <= DW_REL * np.abs(wb).max(), f"call {call}: {name}"
+    assert eng.engram_read_device_error() == 0
+
+
+def test_noalloc_rejects_oversize_hidden_size():
+    # one row of H > 65536 values: refused with a status, nothing launched
+    t = _inputs(220, 2, 64)
+    st = eng.lib().engram_gate_bwd_noalloc(
+        t["g"].data_ptr(), t["x"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(),
+        t["wh"].data_ptr(), t["we"].data_ptr(), 1, 65544, 1e-6, 0.125, t["x"].data_ptr(),
+        t["k"].data_ptr(), t["v"].data_ptr(), t["x"].data_ptr(), t["k"].data_ptr(),
+        torch.cuda.current_stream().cuda_stream)
+    assert st in (1, 2)
+    torch.cuda.synchronize()
     assert eng.engram_read_device_error() == 0
 
 
