@@ -345,7 +345,7 @@ def run_ours(args):
 
     # Cache-cold control for the gather: the same hash_gather launch on ids drawn
     # uniformly over the vocabulary (no hot rows), L2 flushed before each launch.
-    uniform = None
+    uniform = l2_state = None
     if args.uniform_control and rank == 0 and w.vocab > 0:
         from engram_conditional_memory_hash_b200 import inputs as _inp
         utok = torch.from_numpy(_inp.uniform_ids(w.seed, 99, (w.B, w.S), 0, w.vocab)).to(dev)
@@ -367,6 +367,29 @@ def run_ours(args):
                 ts.append(e0.elapsed_time(e1))
         uniform = kernel_entry(float(np.median(ts)) * 1e3, ab["hash_gather"], peak)
         uniform["ids"] = f"uniform over [0, {w.vocab}), L2 flushed before each launch"
+        # The step's own launch (its Zipf ids) after L2 was filled with clean
+        # lines (a read of a buffer twice its size) and with dirty ones (a
+        # write): inside the step the launch follows the gate backward, whose
+        # last output writes are still in L2 and are written back meanwhile.
+        after = {}
+        for mode in ("clean", "dirty"):
+            ts = []
+            for it in range(13):
+                if mode == "clean":
+                    flush.max()
+                else:
+                    flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                eng.engram_hash_gather(buf0.tokens, hin["multipliers"], hin["ngram_n"],
+                                       hin["table_sizes"], tables, pad_id=hin["pad_id"],
+                                       idx_out=uidx, rows_out=urows, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                if it >= 3:
+                    ts.append(e0.elapsed_time(e1))
+            after[mode] = kernel_entry(float(np.median(ts)) * 1e3, ab["hash_gather"], peak)
+        l2_state = after
         del flush, uidx, urows
 
     # Gather backward (the transpose of the gather: row gradients summed into
@@ -553,6 +576,7 @@ def run_ours(args):
                 world * T / ((per_kernel_ms["gate_fwd"] + per_kernel_ms["gate_bwd"]) / 1e3), 1),
             "kernels": kern,
             "hash_gather_uniform_ids": uniform,
+            "hash_gather_after_l2": l2_state,
             "gather_bwd": gbwd,
             "configs": configs,
             "roofline": roof,

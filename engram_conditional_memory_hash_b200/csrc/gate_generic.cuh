@@ -8,7 +8,9 @@
 //
 // One CTA per token at a time (persistent: CTA c handles tokens c, c+G, ...),
 // two passes over the token's rows, consecutive threads on consecutive
-// columns: the first accumulates the statistics (fp32 sums of squares and of
+// columns, each thread loading kGenBatch vectors of every row it needs before
+// it uses any (so that many loads are in flight per thread): the first pass
+// accumulates the statistics (fp32 sums of squares and of
 // g*v, the dot product sum x k w in fp64 exactly as the tuned kernels do), a
 // fixed-order block reduction combines them, the per-token scalars come from
 // the same gate_scalars(), and the second pass reads the rows again (from L2:
@@ -118,6 +120,38 @@ __device__ __forceinline__ void for_columns(const void *row, int H, F &&f)
     if (tail + (int)threadIdx.x < H) f(tail + (int)threadIdx.x, false);
 }
 
+// The same visit with the body vectors in batches of kGenBatch per thread:
+// load(b, j) for the batch's vectors (b = 0..kGenBatch-1, column j) first, so
+// that all of their loads are in flight together, then use(b, j) for each in
+// order (the order in which for_columns would visit them).  col(j) handles a
+// single column (head, tail, or every column without VEC).
+#ifndef ENGRAM_GEN_BATCH
+#define ENGRAM_GEN_BATCH 4
+#endif
+constexpr int kGenBatch = ENGRAM_GEN_BATCH;
+
+template <bool VEC, typename FC, typename FL, typename FU>
+__device__ __forceinline__ void for_columns_batched(const void *row, int H, FC &&col, FL &&load, FU &&use)
+{
+    if (!VEC) {
+        for (int j = threadIdx.x; j < H; j += kGenThreads) col(j);
+        return;
+    }
+    const int head = row_head(row, H);
+    const int nvec = (H - head) >> 3;
+    const int tail = head + 8 * nvec;
+    if ((int)threadIdx.x < head) col((int)threadIdx.x);
+    for (int i0 = threadIdx.x; i0 < nvec; i0 += kGenBatch * kGenThreads) {
+#pragma unroll
+        for (int b = 0; b < kGenBatch; ++b)
+            if (i0 + b * kGenThreads < nvec) load(b, head + 8 * (i0 + b * kGenThreads));
+#pragma unroll
+        for (int b = 0; b < kGenBatch; ++b)
+            if (i0 + b * kGenThreads < nvec) use(b, head + 8 * (i0 + b * kGenThreads));
+    }
+    if (tail + (int)threadIdx.x < H) col(tail + (int)threadIdx.x);
+}
+
 template <bool VEC>
 __global__ void __launch_bounds__(kGenThreads)
 gate_generic_fwd_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ k,
@@ -133,12 +167,24 @@ gate_generic_fwd_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16
         __nv_bfloat16 *orow = out + t * H;
         float px = 0.f, pk = 0.f;
         double pa = 0.0;
-        for_columns<VEC>(xr, H, [&](int j, bool vec) {
-            if (vec) {
+        uint4 xq[kGenBatch], kq[kGenBatch];
+        for_columns_batched<VEC>(
+            xr, H,
+            [&](int j) {
+                const float xv = bf(xr + j), kv = bf(kr + j);
+                px = fmaf(xv, xv, px);
+                pk = fmaf(kv, kv, pk);
+                pa = fma((double)(xv * kv), (double)wcol(wh, we, j), pa);
+            },
+            [&](int b, int j) {
+                xq[b] = *reinterpret_cast<const uint4 *>(xr + j);
+                kq[b] = *reinterpret_cast<const uint4 *>(kr + j);
+            },
+            [&](int b, int j) {
                 float2 xf[4], kf[4];
                 float w[8];
-                unpack4x2(*reinterpret_cast<const uint4 *>(xr + j), xf);
-                unpack4x2(*reinterpret_cast<const uint4 *>(kr + j), kf);
+                unpack4x2(xq[b], xf);
+                unpack4x2(kq[b], kf);
                 wvec(wh, we, j, w);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -147,30 +193,28 @@ gate_generic_fwd_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16
                     pa = fma((double)(xf[e].x * kf[e].x), (double)w[2 * e], pa);
                     pa = fma((double)(xf[e].y * kf[e].y), (double)w[2 * e + 1], pa);
                 }
-            } else {
-                const float xv = bf(xr + j), kv = bf(kr + j);
-                px = fmaf(xv, xv, px);
-                pk = fmaf(kv, kv, pk);
-                pa = fma((double)(xv * kv), (double)wcol(wh, we, j), pa);
-            }
-        });
+            });
         float4 r;
         double A;
         gen_block_reduce(px, pk, 0.f, pa, red, redd, r, A);
         const GateScalars c = gate_scalars(r.x, r.y, A, inv_h, eps, scalar);
-        for_columns<VEC>(xr, H, [&](int j, bool vec) {
-            if (vec) {
+        uint4 vq[kGenBatch];
+        for_columns_batched<VEC>(
+            xr, H,
+            [&](int j) { orow[j] = __float2bfloat16_rn(fmaf(c.gate, bf(vr + j), bf(xr + j))); },
+            [&](int b, int j) {
+                xq[b] = *reinterpret_cast<const uint4 *>(xr + j);
+                vq[b] = *reinterpret_cast<const uint4 *>(vr + j);
+            },
+            [&](int b, int j) {
                 float2 xf[4], vf[4], of[4];
-                unpack4x2(*reinterpret_cast<const uint4 *>(xr + j), xf);
-                unpack4x2(*reinterpret_cast<const uint4 *>(vr + j), vf);
+                unpack4x2(xq[b], xf);
+                unpack4x2(vq[b], vf);
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     of[e] = make_float2(fmaf(c.gate, vf[e].x, xf[e].x), fmaf(c.gate, vf[e].y, xf[e].y));
                 __stcs(reinterpret_cast<uint4 *>(orow + j), pack4x2(of));
-            } else {
-                orow[j] = __float2bfloat16_rn(fmaf(c.gate, bf(vr + j), bf(xr + j)));
-            }
-        });
+            });
         if (threadIdx.x == 0 && gate != nullptr) gate[t] = c.gate;
     }
 }
@@ -195,14 +239,29 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
         const __nv_bfloat16 *gr = gout + t * H, *xr = x + t * H, *kr = k + t * H, *vr = v + t * H;
         float px = 0.f, pk = 0.f, pg = 0.f;
         double pa = 0.0;
-        for_columns<VEC>(xr, H, [&](int j, bool vec) {
-            if (vec) {
+        uint4 gq[kGenBatch], xq[kGenBatch], kq[kGenBatch], vq[kGenBatch];
+        for_columns_batched<VEC>(
+            xr, H,
+            [&](int j) {
+                const float xv = bf(xr + j), kv = bf(kr + j);
+                px = fmaf(xv, xv, px);
+                pk = fmaf(kv, kv, pk);
+                pg = fmaf(bf(gr + j), bf(vr + j), pg);
+                pa = fma((double)(xv * kv), (double)wcol(wh, we, j), pa);
+            },
+            [&](int b, int j) {
+                gq[b] = *reinterpret_cast<const uint4 *>(gr + j);
+                xq[b] = *reinterpret_cast<const uint4 *>(xr + j);
+                kq[b] = *reinterpret_cast<const uint4 *>(kr + j);
+                vq[b] = *reinterpret_cast<const uint4 *>(vr + j);
+            },
+            [&](int b, int j) {
                 float2 gf[4], xf[4], kf[4], vf[4];
                 float w[8];
-                unpack4x2(*reinterpret_cast<const uint4 *>(gr + j), gf);
-                unpack4x2(*reinterpret_cast<const uint4 *>(xr + j), xf);
-                unpack4x2(*reinterpret_cast<const uint4 *>(kr + j), kf);
-                unpack4x2(*reinterpret_cast<const uint4 *>(vr + j), vf);
+                unpack4x2(gq[b], gf);
+                unpack4x2(xq[b], xf);
+                unpack4x2(kq[b], kf);
+                unpack4x2(vq[b], vf);
                 wvec(wh, we, j, w);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -212,14 +271,7 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
                     pa = fma((double)(xf[e].x * kf[e].x), (double)w[2 * e], pa);
                     pa = fma((double)(xf[e].y * kf[e].y), (double)w[2 * e + 1], pa);
                 }
-            } else {
-                const float xv = bf(xr + j), kv = bf(kr + j);
-                px = fmaf(xv, xv, px);
-                pk = fmaf(kv, kv, pk);
-                pg = fmaf(bf(gr + j), bf(vr + j), pg);
-                pa = fma((double)(xv * kv), (double)wcol(wh, we, j), pa);
-            }
-        });
+            });
         float4 r;
         double A;
         gen_block_reduce(px, pk, pg, pa, red, redd, r, A);
@@ -232,13 +284,27 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
         const float c2 = dd * c.d * c.rx * c.rx * inv_h;
         const float c3 = dd * c.d * c.rk * c.rk * inv_h;
         __nv_bfloat16 *dxr = dx + t * H, *dkr = dk + t * H, *dvr = dv + t * H;
-        for_columns<VEC>(xr, H, [&](int j, bool vec) {
-            if (vec) {
+        for_columns_batched<VEC>(
+            xr, H,
+            [&](int j) {
+                const float gv = bf(gr + j), xv = bf(xr + j), kv = bf(kr + j);
+                const float cw = c1 * wcol(wh, we, j);
+                dxr[j] = __float2bfloat16_rn(fmaf(-c2, xv, fmaf(cw, kv, gv)));
+                dkr[j] = __float2bfloat16_rn(fmaf(-c3, kv, cw * xv));
+                dvr[j] = __float2bfloat16_rn(c.gate * gv);
+                acc[j] = fmaf(c1, xv * kv, acc[j]);
+            },
+            [&](int bb, int j) {
+                gq[bb] = *reinterpret_cast<const uint4 *>(gr + j);
+                xq[bb] = *reinterpret_cast<const uint4 *>(xr + j);
+                kq[bb] = *reinterpret_cast<const uint4 *>(kr + j);
+            },
+            [&](int bb, int j) {
                 float2 gf[4], xf[4], kf[4], a[4], b[4], cv[4];
                 float w[8], pr[8];
-                unpack4x2(*reinterpret_cast<const uint4 *>(gr + j), gf);
-                unpack4x2(*reinterpret_cast<const uint4 *>(xr + j), xf);
-                unpack4x2(*reinterpret_cast<const uint4 *>(kr + j), kf);
+                unpack4x2(gq[bb], gf);
+                unpack4x2(xq[bb], xf);
+                unpack4x2(kq[bb], kf);
                 wvec(wh, we, j, w);
                 const bool acc4 = (reinterpret_cast<uintptr_t>(acc + j) & 15u) == 0;
                 if (acc4) {
@@ -270,15 +336,7 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
                 __stcs(reinterpret_cast<uint4 *>(dxr + j), pack4x2(a));
                 __stcs(reinterpret_cast<uint4 *>(dkr + j), pack4x2(b));
                 __stcs(reinterpret_cast<uint4 *>(dvr + j), pack4x2(cv));
-            } else {
-                const float gv = bf(gr + j), xv = bf(xr + j), kv = bf(kr + j);
-                const float cw = c1 * wcol(wh, we, j);
-                dxr[j] = __float2bfloat16_rn(fmaf(-c2, xv, fmaf(cw, kv, gv)));
-                dkr[j] = __float2bfloat16_rn(fmaf(-c3, kv, cw * xv));
-                dvr[j] = __float2bfloat16_rn(c.gate * gv);
-                acc[j] = fmaf(c1, xv * kv, acc[j]);
-            }
-        });
+            });
     }
     if (acc != prow) {
         __syncthreads();
