@@ -137,7 +137,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20", "-i", str(self.idx)],
+                 "-lms", "10", "-i", str(self.idx)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -591,7 +591,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-GATHER_BWD_LAUNCHES = 12
+GATHER_BWD_LAUNCHES = 13
 
 
 def measure_config(name: str, dev, peak: float, iters: int = 20, warmup: int = 3) -> dict:

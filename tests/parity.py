@@ -7,9 +7,11 @@ Tolerances (the same for every test):
   ref the fp64 oracle value (2^-8 |ref| bounds the final rounding to bf16);
 * the fp32 gate: |gpu - ref| <= 1e-4;
 * dwh, dwe: max |gpu - ref| <= 1e-3 max |ref|.
-Tokens whose signed_sqrt argument is tiny (|s| < 1e-4) amplify the fp32
-rounding of s through 1/(2 sqrt|s|); their dx/dk rows are held to 1e-2 of the
-row's largest |ref| instead (see ill_conditioned()).
+Tokens whose signed_sqrt argument is small (1e-6 <= |s| < 1e-4) amplify the
+fp32 rounding of s through 1/(2 sqrt|s|); their dx/dk rows are held to 1e-2 of
+the row's largest |ref| instead (see ill_conditioned()).  Below 1e-6 the
+derivative's clamp makes the factor a constant, so those tokens keep the
+strict bound.
 """
 import numpy as np
 import torch
@@ -19,6 +21,7 @@ BF16_REL = 2.0 ** -8
 GATE_ABS = 1e-4
 DW_REL = 1e-3
 ILL_S = 1e-4
+CLAMP_S = 1e-6
 
 
 def to_dev_bf16(a: np.ndarray, dev="cuda") -> torch.Tensor:
@@ -62,7 +65,8 @@ def assert_dw_close(name, got: torch.Tensor, want: np.ndarray):
 
 
 def ill_conditioned(s_ref: np.ndarray) -> np.ndarray:
-    return np.abs(s_ref) < ILL_S
+    a = np.abs(s_ref)
+    return (a >= CLAMP_S) & (a < ILL_S)
 
 
 def check_gate_blockwise(o, gi, res, eps, blk=2048, forward=True):
