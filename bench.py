@@ -645,6 +645,9 @@ def measure_config(name: str, dev, peak: float, iters: int = 20, warmup: int = 3
     flush_l2 = name in ("tiny", "hash_gather")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush_l2 else None
     times = {n: [] for n in names}
+    evs = []
+    # every iteration enqueued back to back (no host synchronisation between
+    # them), events between the launches
     for it in range(warmup + iters):
         if flush is not None:
             flush.zero_()
@@ -653,10 +656,12 @@ def measure_config(name: str, dev, peak: float, iters: int = 20, warmup: int = 3
         for i, n in enumerate(names):
             calls[n]()
             ev[i + 1].record(stream)
-        torch.cuda.synchronize(dev)
         if it >= warmup:
-            for i, n in enumerate(names):
-                times[n].append(ev[i].elapsed_time(ev[i + 1]))
+            evs.append(ev)
+    torch.cuda.synchronize(dev)
+    for ev in evs:
+        for i, n in enumerate(names):
+            times[n].append(ev[i].elapsed_time(ev[i + 1]))
     assert eng.engram_read_device_error() == 0
     ab = algorithmic_bytes(T, max(H, 1), w.L, w.J, w.D, G)
     kern = {n: kernel_entry(float(np.median(times[n])) * 1e3, ab[n], peak) for n in names}
@@ -665,7 +670,8 @@ def measure_config(name: str, dev, peak: float, iters: int = 20, warmup: int = 3
            "tokens_per_s": round(T / (total_us / 1e6), 1),
            "l2": "flushed before every iteration" if flush_l2 else
                  "inputs larger than L2; iterations back to back",
-           "timing": f"median of {iters} iterations after {warmup}, CUDA events per launch"}
+           "timing": f"median of {iters} iterations after {warmup}, enqueued back to back, "
+                     "CUDA events between the launches"}
     if w.has_hash:
         res["tables"] = f"{w.L * w.J} x ~{w.prime_base} rows x {w.D} bf16, ids {w.ids}"
     return res

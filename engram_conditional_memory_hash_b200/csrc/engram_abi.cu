@@ -80,15 +80,18 @@ engram_status_t device_info(DeviceInfo *out)
 constexpr int kGateMaxH = 8192;
 
 // Launch shape of the gate kernels, chosen by timing launch shapes on B200 at
-// H = 4096 and 7168: the forward runs 2 CTAs per SM of at most 256 threads
-// (4 vectors per thread at H = 7168); the backward, whose registers hold four
-// rows' worth of vectors plus the weight-gradient accumulators, runs one CTA
-// per SM with 2 vectors per thread.  Overridable at compile time.
+// H = 4096 and 7168: the forward runs CTAs of at most 256 threads (4 vectors
+// per thread at H = 7168), as many per SM as registers allow up to 4, with the
+// shared memory split between them (2 CTAs at both sizes; at H = 4096 that
+// leaves 2 pipeline stages each, 86.5 us per forward of 16384 tokens against
+// 96.9 with 4 stages when the cap was 2 CTAs); the backward, whose registers
+// hold four rows' worth of vectors plus the weight-gradient accumulators, runs
+// one CTA per SM with 2 vectors per thread.  Overridable at compile time.
 #ifndef ENGRAM_FWD_TARGET_THREADS
 #define ENGRAM_FWD_TARGET_THREADS 256
 #endif
 #ifndef ENGRAM_FWD_MAX_CTAS
-#define ENGRAM_FWD_MAX_CTAS 2
+#define ENGRAM_FWD_MAX_CTAS 4
 #endif
 #ifndef ENGRAM_BWD_VEC
 #define ENGRAM_BWD_VEC 2
@@ -229,27 +232,34 @@ bool same_phase(std::initializer_list<const void *> ptrs)
 // CTAs of a generic gate kernel: as many as the SMs hold at once (one wave),
 // never more than tokens.
 template <typename K>
-engram_status_t generic_grid(const DeviceInfo &d, int64_t T, K kernel, size_t smem, int64_t *grid)
+engram_status_t generic_grid(const DeviceInfo &d, int64_t T, int H, K kernel, size_t smem, int64_t *grid)
 {
     int n = 0;
-    engram_status_t st = occupancy(kernel, engram::kGenThreads, smem, &n);
+    engram_status_t st = occupancy(kernel, engram::gen_threads(H), smem, &n);
     if (st != ENGRAM_OK) return st;
     *grid = std::max<int64_t>(1, std::min<int64_t>(T, (int64_t)d.sms * std::max(n, 1)));
     return ENGRAM_OK;
 }
 
 // Dynamic shared memory of the generic backward: its partial row, when it fits.
-size_t generic_bwd_smem(int H) { return H <= engram::kGenSmemPartial ? (size_t)H * 4 : 0; }
+size_t generic_bwd_smem(int H) { return H <= engram::kGenSmemPartial ? (size_t)(H + 8) * 4 : 0; }
 
 // Partial rows (CTAs) of the generic backward: one wave of the kernel variant
-// with the fewer resident CTAs per SM.
+// with the fewer resident CTAs per SM, rounded down to a multiple of
+// 8 / gcd(H, 8) so that G * H is a multiple of 8: then every token row of a
+// CTA starts at the same offset from a 16-byte boundary (rows c, c + G, ...
+// are G * H values apart) and the CTA's partial row can be laid out for
+// 16-byte access (see gate_generic_bwd_kernel).
 engram_status_t generic_bwd_grid(const DeviceInfo &d, int64_t T, int H, int64_t *grid)
 {
     int64_t a = 0, b = 0;
     const size_t smem = generic_bwd_smem(H);
-    engram_status_t st = generic_grid(d, T, engram::gate_generic_bwd_kernel<true>, smem, &a);
-    if (st == ENGRAM_OK) st = generic_grid(d, T, engram::gate_generic_bwd_kernel<false>, smem, &b);
-    *grid = std::min(a, b);
+    engram_status_t st = generic_grid(d, T, H, engram::gate_generic_bwd_kernel<true>, smem, &a);
+    if (st == ENGRAM_OK) st = generic_grid(d, T, H, engram::gate_generic_bwd_kernel<false>, smem, &b);
+    int64_t g = std::min(a, b);
+    const int64_t m = 8 / ((H & 7) == 0 ? 8 : (H & 3) == 0 ? 4 : (H & 1) == 0 ? 2 : 1);
+    if (g >= m) g -= g % m;
+    *grid = g;
     return st;
 }
 
@@ -288,21 +298,40 @@ engram_status_t launch_gate_bwd_tuned(const DeviceInfo &dev, const void *grad_ou
     engram_status_t st = gate_bwd_plan(dev, H, &g);
     if (st != ENGRAM_OK) return st;
     const engram::ReduceGroups grp = engram::reduce_groups(G);
+    // CTAs of the fused tail that may wait for the others: half of those the
+    // GPU holds at once
+    const int kmax = std::max(1, dev.sms * g.ctas_per_sm / 2);
     auto args = [&](auto kern) -> engram_status_t {
+        // the plan sized the launch on the plain kernel; the fused variant
+        // needs the same shared-memory opt-in
+        if (tickets != nullptr) {
+            const cudaError_t ea =
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
+            if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute");
+        }
         kern<<<(unsigned)G, g.threads, g.smem, s>>>(
             static_cast<const uint4 *>(grad_out), static_cast<const uint4 *>(x),
             static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<const uint4 *>(wh),
             static_cast<const uint4 *>(we), T, H, eps, scalar, static_cast<uint4 *>(dx),
-            static_cast<uint4 *>(dk), static_cast<uint4 *>(dv), w_partial, g.nstage, tickets, grp, dwh,
+            static_cast<uint4 *>(dk), static_cast<uint4 *>(dv), w_partial, g.nstage, tickets, grp, kmax, dwh,
             dwe);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "gate_bwd launch");
         return ENGRAM_OK;
     };
-    if (g.maxv == 2 && g.threads <= kBwdNarrowThreads) return args(engram::gate_bwd_kernel<2, kBwdNarrowThreads>);
-    return g.maxv == 1 ? args(engram::gate_bwd_kernel<1>)
-         : g.maxv == 2 ? args(engram::gate_bwd_kernel<2>)
-                       : args(engram::gate_bwd_kernel<4>);
+    using engram::gate_bwd_kernel;
+    constexpr int M1 = engram::gate_max_threads(1), M2 = engram::gate_max_threads(2),
+                  M4 = engram::gate_max_threads(4);
+    if (tickets != nullptr) {
+        if (g.maxv == 2 && g.threads <= kBwdNarrowThreads) return args(gate_bwd_kernel<2, kBwdNarrowThreads, true>);
+        return g.maxv == 1 ? args(gate_bwd_kernel<1, M1, true>)
+             : g.maxv == 2 ? args(gate_bwd_kernel<2, M2, true>)
+                           : args(gate_bwd_kernel<4, M4, true>);
+    }
+    if (g.maxv == 2 && g.threads <= kBwdNarrowThreads) return args(gate_bwd_kernel<2, kBwdNarrowThreads>);
+    return g.maxv == 1 ? args(gate_bwd_kernel<1>)
+         : g.maxv == 2 ? args(gate_bwd_kernel<2>)
+                       : args(gate_bwd_kernel<4>);
 }
 
 }  // namespace
@@ -433,8 +462,8 @@ engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, con
         auto kern = same_phase({x, k, v, out}) ? engram::gate_generic_fwd_kernel<true>
                                                : engram::gate_generic_fwd_kernel<false>;
         int64_t grid = 0;
-        if ((st = generic_grid(dev, T, kern, 0, &grid)) != ENGRAM_OK) return st;
-        kern<<<(unsigned)grid, engram::kGenThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        if ((st = generic_grid(dev, T, H, kern, 0, &grid)) != ENGRAM_OK) return st;
+        kern<<<(unsigned)grid, engram::gen_threads(H), 0, reinterpret_cast<cudaStream_t>(stream)>>>(
             static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(k),
             static_cast<const __nv_bfloat16 *>(v), static_cast<const __nv_bfloat16 *>(wh),
             static_cast<const __nv_bfloat16 *>(we), T, H, eps, scalar, static_cast<__nv_bfloat16 *>(out),
@@ -508,9 +537,9 @@ engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void 
                                                                  : engram::gate_generic_bwd_kernel<false>;
         const size_t smem = generic_bwd_smem(H);
         cudaError_t e0 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              (int)(engram::kGenSmemPartial * 4));
+                                              (int)((engram::kGenSmemPartial + 8) * 4));
         if (e0 != cudaSuccess) return cuda_fail(e0, "cudaFuncSetAttribute");
-        kern<<<(unsigned)G, engram::kGenThreads, smem, s>>>(
+        kern<<<(unsigned)G, engram::gen_threads(H), smem, s>>>(
             static_cast<const __nv_bfloat16 *>(grad_out), static_cast<const __nv_bfloat16 *>(x),
             static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v),
             static_cast<const __nv_bfloat16 *>(wh), static_cast<const __nv_bfloat16 *>(we), T, H, eps, scalar,

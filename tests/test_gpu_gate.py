@@ -125,7 +125,7 @@ def test_deterministic(oracle_lib):
 
 
 @pytest.mark.parametrize("T,H", [(3, 1), (5, 7), (129, 100), (40, 1001), (17, 8200), (9, 16384),
-                                 (3, 65536)])
+                                 (3, 65536), (600, 7169), (300, 2050)])
 def test_generic_hidden_sizes(oracle_lib, T, H):
     # H not a multiple of 8 or above 8192: the generic kernels; every output
     # against the oracle, and G covering more and fewer CTAs than tokens
