@@ -238,6 +238,24 @@ def gather_bwd_bytes(T: int, L: int, J: int, D: int, unique_rows: int) -> int:
     return T * L * J * (8 + 2 * D) + unique_rows * 2 * 4 * D
 
 
+class L2Flush:
+    """Empties L2 between timed launches: writes a buffer twice the L2 size,
+    then reads another one, so that the lines the write left dirty are
+    written back before the timed launch starts (which then begins on a cold,
+    clean L2)."""
+
+    WHAT = "a 252 MB buffer written, then another 252 MB read"
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.max()
+
+
 def time_calls(call, stream, dev, warmup: int, calls: int) -> float:
     """Microseconds per call of `call` (which enqueues GPU work on `stream`):
     `warmup` calls, then `calls` calls enqueued back to back between two CUDA
@@ -349,13 +367,13 @@ def run_ours(args):
     if args.uniform_control and rank == 0 and w.vocab > 0:
         from engram_conditional_memory_hash_b200 import inputs as _inp
         utok = torch.from_numpy(_inp.uniform_ids(w.seed, 99, (w.B, w.S), 0, w.vocab)).to(dev)
-        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        flush = L2Flush(dev)
         # its own outputs: the step's indices in buf0 stay those of the step's
         # tokens (the gather backward below runs on them)
         uidx, urows = torch.empty_like(buf0.idx), torch.empty_like(buf0.rows)
         ts = []
         for it in range(13):
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             eng.engram_hash_gather(utok, hin["multipliers"], hin["ngram_n"], hin["table_sizes"],
@@ -366,19 +384,20 @@ def run_ours(args):
             if it >= 3:
                 ts.append(e0.elapsed_time(e1))
         uniform = kernel_entry(float(np.median(ts)) * 1e3, ab["hash_gather"], peak)
-        uniform["ids"] = f"uniform over [0, {w.vocab}), L2 flushed before each launch"
-        # The step's own launch (its Zipf ids) after L2 was filled with clean
-        # lines (a read of a buffer twice its size) and with dirty ones (a
-        # write): inside the step the launch follows the gate backward, whose
+        uniform["ids"] = (f"uniform over [0, {w.vocab}), L2 flushed before each launch "
+                          f"({L2Flush.WHAT})")
+        # The step's own launch (its Zipf ids) after L2 was emptied (clean) and
+        # after it was filled with dirty lines (a write of a buffer twice its
+        # size): inside the step the launch follows the gate backward, whose
         # last output writes are still in L2 and are written back meanwhile.
         after = {}
         for mode in ("clean", "dirty"):
             ts = []
             for it in range(13):
                 if mode == "clean":
-                    flush.max()
+                    flush()
                 else:
-                    flush.zero_()
+                    flush.w.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 eng.engram_hash_gather(buf0.tokens, hin["multipliers"], hin["ngram_n"],
@@ -643,14 +662,14 @@ def measure_config(name: str, dev, peak: float, iters: int = 20, warmup: int = 3
                 dv=dv, w_partial=part, tickets=tickets, dwh=dw[0], dwe=dw[1], stream=stream)
     names = [n for n in engram_step.LAUNCHES if n in calls]
     flush_l2 = name in ("tiny", "hash_gather")
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush_l2 else None
+    flush = L2Flush(dev) if flush_l2 else None
     times = {n: [] for n in names}
     evs = []
     # every iteration enqueued back to back (no host synchronisation between
     # them), events between the launches
     for it in range(warmup + iters):
         if flush is not None:
-            flush.zero_()
+            flush()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
         ev[0].record(stream)
         for i, n in enumerate(names):
@@ -668,7 +687,7 @@ def measure_config(name: str, dev, peak: float, iters: int = 20, warmup: int = 3
     total_us = sum(k["us"] for k in kern.values())
     res = {"T": T, "H": H or None, "launches": names, "kernels": kern,
            "tokens_per_s": round(T / (total_us / 1e6), 1),
-           "l2": "flushed before every iteration" if flush_l2 else
+           "l2": f"flushed before every iteration ({L2Flush.WHAT})" if flush_l2 else
                  "inputs larger than L2; iterations back to back",
            "timing": f"median of {iters} iterations after {warmup}, enqueued back to back, "
                      "CUDA events between the launches"}

@@ -11,7 +11,9 @@
 #include <cstdio>
 #include <cstring>
 #include <initializer_list>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "engram.h"
 
@@ -43,6 +45,7 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Per-device facts used to size the launches, read once per device.
 struct DeviceInfo {
+    int ordinal = 0;
     int sms = 0;
     int smem_optin = 0;     // largest dynamic shared memory a CTA may opt into
     int smem_per_sm = 0;
@@ -62,6 +65,7 @@ engram_status_t device_info(DeviceInfo *out)
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!g_dev_ready[dev]) {
         DeviceInfo d;
+        d.ordinal = dev;
         if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
             (e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
                 cudaSuccess ||
@@ -112,10 +116,16 @@ struct GateLaunch {
 };
 
 // Resident CTAs per SM of `kernel` with the given block and shared memory.
+// The kernel's shared-memory opt-in is raised to `smem` and never lowered, so
+// that a launch sized by an earlier (cached) plan stays valid.
 template <typename K>
 engram_status_t occupancy(K kernel, int threads, size_t smem, int *n)
 {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+    if ((size_t)fa.maxDynamicSharedSizeBytes < smem)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, kernel, threads, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
@@ -193,6 +203,32 @@ engram_status_t gate_bwd_plan(const DeviceInfo &d, int H, GateLaunch *g)
                      engram::gate_bwd_kernel<2>, engram::gate_bwd_kernel<4>, g);
 }
 
+// The plans, computed once per device, hidden size and direction: planning
+// sets the kernels' shared-memory attributes and queries the occupancy API,
+// host calls that cost time on every launch otherwise (and setting an
+// attribute of a kernel that is still running can make the host wait for it,
+// leaving the GPU idle between calls).  The fused backward's attribute is set
+// here too, once.
+std::mutex g_plan_mutex;
+std::map<std::pair<int, int>, GateLaunch> g_plans;   // (ordinal * 2 + direction, H)
+
+engram_status_t set_fused_bwd_attribute(const GateLaunch &g);
+
+engram_status_t cached_gate_plan(const DeviceInfo &d, int H, bool backward, GateLaunch *g)
+{
+    const std::pair<int, int> key(d.ordinal * 2 + (backward ? 1 : 0), H);
+    std::lock_guard<std::mutex> lock(g_plan_mutex);
+    auto it = g_plans.find(key);
+    if (it != g_plans.end()) {
+        *g = it->second;
+        return ENGRAM_OK;
+    }
+    engram_status_t st = backward ? gate_bwd_plan(d, H, g) : gate_fwd_plan(d, H, g);
+    if (st == ENGRAM_OK && backward) st = set_fused_bwd_attribute(*g);
+    if (st == ENGRAM_OK) g_plans.emplace(key, *g);
+    return st;
+}
+
 engram_status_t check_gate_common(int64_t T, int32_t H, float eps, float scalar)
 {
     if (T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "T=%lld < 0", (long long)T);
@@ -229,6 +265,52 @@ bool same_phase(std::initializer_list<const void *> ptrs)
     return true;
 }
 
+// The generic kernel variant for rows of H values: VEC (token tensors share
+// their offset from a 16-byte boundary), SHIFT (see shifted_rows) and the
+// block size gen_threads(H).
+using GenFwdKernel = void (*)(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *,
+                              const __nv_bfloat16 *, const __nv_bfloat16 *, int64_t, int, float, float,
+                              __nv_bfloat16 *, float *);
+using GenBwdKernel = void (*)(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *,
+                              const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, int64_t, int,
+                              float, float, __nv_bfloat16 *, __nv_bfloat16 *, __nv_bfloat16 *, float *);
+
+template <int NT>
+GenFwdKernel gen_fwd_variant(bool vec, bool shift)
+{
+    using namespace engram;
+    return !vec ? gate_generic_fwd_kernel<false, false, NT>
+         : shift ? gate_generic_fwd_kernel<true, true, NT> : gate_generic_fwd_kernel<true, false, NT>;
+}
+
+template <int NT>
+GenBwdKernel gen_bwd_variant(bool vec, bool shift)
+{
+    using namespace engram;
+    return !vec ? gate_generic_bwd_kernel<false, false, NT>
+         : shift ? gate_generic_bwd_kernel<true, true, NT> : gate_generic_bwd_kernel<true, false, NT>;
+}
+
+GenFwdKernel gen_fwd_kernel(int H, bool vec, bool shift)
+{
+    const int nt = engram::gen_threads(H);
+    return nt == 64 ? gen_fwd_variant<64>(vec, shift)
+         : nt == 128 ? gen_fwd_variant<128>(vec, shift) : gen_fwd_variant<256>(vec, shift);
+}
+
+GenBwdKernel gen_bwd_kernel(int H, bool vec, bool shift)
+{
+    const int nt = engram::gen_threads(H);
+    return nt == 64 ? gen_bwd_variant<64>(vec, shift)
+         : nt == 128 ? gen_bwd_variant<128>(vec, shift) : gen_bwd_variant<256>(vec, shift);
+}
+
+// Whether some token row of a tensor starting at `x` with rows of H values has
+// its 16-byte vectors off the 16-byte boundaries of wh and we (odd rows, or a
+// tensor past a boundary): the generic kernels then build the fused weight
+// from aligned chunks (SHIFT).
+bool shifted_rows(int H, const void *x) { return (H % 8) != 0 || !aligned(x, 16); }
+
 // CTAs of a generic gate kernel: as many as the SMs hold at once (one wave),
 // never more than tokens.
 template <typename K>
@@ -254,9 +336,11 @@ engram_status_t generic_bwd_grid(const DeviceInfo &d, int64_t T, int H, int64_t 
 {
     int64_t a = 0, b = 0;
     const size_t smem = generic_bwd_smem(H);
-    engram_status_t st = generic_grid(d, T, H, engram::gate_generic_bwd_kernel<true>, smem, &a);
-    if (st == ENGRAM_OK) st = generic_grid(d, T, H, engram::gate_generic_bwd_kernel<false>, smem, &b);
-    int64_t g = std::min(a, b);
+    int64_t c = 0;
+    engram_status_t st = generic_grid(d, T, H, gen_bwd_kernel(H, true, true), smem, &a);
+    if (st == ENGRAM_OK) st = generic_grid(d, T, H, gen_bwd_kernel(H, true, false), smem, &b);
+    if (st == ENGRAM_OK) st = generic_grid(d, T, H, gen_bwd_kernel(H, false, false), smem, &c);
+    int64_t g = std::min(std::min(a, b), c);
     const int64_t m = 8 / ((H & 7) == 0 ? 8 : (H & 3) == 0 ? 4 : (H & 1) == 0 ? 2 : 1);
     if (g >= m) g -= g % m;
     *grid = g;
@@ -295,20 +379,13 @@ engram_status_t launch_gate_bwd_tuned(const DeviceInfo &dev, const void *grad_ou
                                       float *dwh, float *dwe, cudaStream_t s)
 {
     GateLaunch g;
-    engram_status_t st = gate_bwd_plan(dev, H, &g);
+    engram_status_t st = cached_gate_plan(dev, H, true, &g);
     if (st != ENGRAM_OK) return st;
     const engram::ReduceGroups grp = engram::reduce_groups(G);
     // CTAs of the fused tail that may wait for the others: half of those the
     // GPU holds at once
     const int kmax = std::max(1, dev.sms * g.ctas_per_sm / 2);
     auto args = [&](auto kern) -> engram_status_t {
-        // the plan sized the launch on the plain kernel; the fused variant
-        // needs the same shared-memory opt-in
-        if (tickets != nullptr) {
-            const cudaError_t ea =
-                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
-            if (ea != cudaSuccess) return cuda_fail(ea, "cudaFuncSetAttribute");
-        }
         kern<<<(unsigned)G, g.threads, g.smem, s>>>(
             static_cast<const uint4 *>(grad_out), static_cast<const uint4 *>(x),
             static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<const uint4 *>(wh),
@@ -332,6 +409,23 @@ engram_status_t launch_gate_bwd_tuned(const DeviceInfo &dev, const void *grad_ou
     return g.maxv == 1 ? args(gate_bwd_kernel<1>)
          : g.maxv == 2 ? args(gate_bwd_kernel<2>)
                        : args(gate_bwd_kernel<4>);
+}
+
+// The shared-memory opt-in of the fused backward variant that a plan launches
+// (the plan itself sized the launch on the plain kernel).
+engram_status_t set_fused_bwd_attribute(const GateLaunch &g)
+{
+    using engram::gate_bwd_kernel;
+    constexpr int M1 = engram::gate_max_threads(1), M2 = engram::gate_max_threads(2),
+                  M4 = engram::gate_max_threads(4);
+    auto set = [&](auto kern) -> engram_status_t {
+        int n = 0;
+        return occupancy(kern, g.threads, g.smem, &n);   // raises the opt-in to g.smem
+    };
+    if (g.maxv == 2 && g.threads <= kBwdNarrowThreads) return set(gate_bwd_kernel<2, kBwdNarrowThreads, true>);
+    return g.maxv == 1 ? set(gate_bwd_kernel<1, M1, true>)
+         : g.maxv == 2 ? set(gate_bwd_kernel<2, M2, true>)
+                       : set(gate_bwd_kernel<4, M4, true>);
 }
 
 }  // namespace
@@ -459,8 +553,7 @@ engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, con
     DeviceInfo dev;
     if ((st = device_info(&dev)) != ENGRAM_OK) return st;
     if (!gate_tuned(H, {x, k, v, wh, we, out})) {
-        auto kern = same_phase({x, k, v, out}) ? engram::gate_generic_fwd_kernel<true>
-                                               : engram::gate_generic_fwd_kernel<false>;
+        const GenFwdKernel kern = gen_fwd_kernel(H, same_phase({x, k, v, out}), shifted_rows(H, x));
         int64_t grid = 0;
         if ((st = generic_grid(dev, T, H, kern, 0, &grid)) != ENGRAM_OK) return st;
         kern<<<(unsigned)grid, engram::gen_threads(H), 0, reinterpret_cast<cudaStream_t>(stream)>>>(
@@ -473,7 +566,7 @@ engram_status_t engram_gate_fwd(const void *x, const void *k, const void *v, con
         return ENGRAM_OK;
     }
     GateLaunch g;
-    if ((st = gate_fwd_plan(dev, H, &g)) != ENGRAM_OK) return st;
+    if ((st = cached_gate_plan(dev, H, false, &g)) != ENGRAM_OK) return st;
     const int64_t grid = std::min<int64_t>(T, (int64_t)dev.sms * g.ctas_per_sm);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     auto args = [&](auto kern) -> engram_status_t {
@@ -505,7 +598,7 @@ int64_t engram_gate_bwd_num_partials(int64_t T, int32_t H)
         return generic_bwd_grid(dev, T, H, &grid) == ENGRAM_OK ? grid : -1;
     }
     GateLaunch g;
-    if (gate_bwd_plan(dev, H, &g) != ENGRAM_OK) return -1;
+    if (cached_gate_plan(dev, H, true, &g) != ENGRAM_OK) return -1;
     const int64_t full = (int64_t)dev.sms * g.ctas_per_sm;
     return std::max<int64_t>(1, std::min<int64_t>(T, full));
 }
@@ -533,12 +626,11 @@ engram_status_t engram_gate_bwd(const void *grad_out, const void *x, const void 
     if ((st = device_info(&dev)) != ENGRAM_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (!gate_tuned(H, {grad_out, x, k, v, wh, we, dx, dk, dv, w_partial})) {
-        auto kern = same_phase({grad_out, x, k, v, dx, dk, dv}) ? engram::gate_generic_bwd_kernel<true>
-                                                                 : engram::gate_generic_bwd_kernel<false>;
+        const GenBwdKernel kern =
+            gen_bwd_kernel(H, same_phase({grad_out, x, k, v, dx, dk, dv}), shifted_rows(H, x));
         const size_t smem = generic_bwd_smem(H);
-        cudaError_t e0 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              (int)((engram::kGenSmemPartial + 8) * 4));
-        if (e0 != cudaSuccess) return cuda_fail(e0, "cudaFuncSetAttribute");
+        int unused = 0;
+        if ((st = occupancy(kern, engram::gen_threads(H), smem, &unused)) != ENGRAM_OK) return st;
         kern<<<(unsigned)G, engram::gen_threads(H), smem, s>>>(
             static_cast<const __nv_bfloat16 *>(grad_out), static_cast<const __nv_bfloat16 *>(x),
             static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v),

@@ -8,10 +8,8 @@
 //
 // One CTA per token at a time (persistent: CTA c handles tokens c, c+G, ...;
 // gen_threads(H) threads, 64 to 256), two passes over the token's rows,
-// consecutive threads on consecutive
-// columns, each thread loading kGenBatch vectors of every row it needs before
-// it uses any (so that many loads are in flight per thread): the first pass
-// accumulates the statistics (fp32 sums of squares and of
+// consecutive threads on consecutive columns: the first pass accumulates the
+// statistics (fp32 sums of squares and of
 // g*v, the dot product sum x k w in fp64 exactly as the tuned kernels do), a
 // fixed-order block reduction combines them, the per-token scalars come from
 // the same gate_scalars(), and the second pass reads the rows again (from L2:
@@ -23,8 +21,12 @@
 // boundary, at most 7), a body of 16-byte vectors (8 columns, one vector per
 // thread at a time) and a tail; head and tail are read element by element.
 // Without VEC every column is read on its own.  The fused weight w = wh * we
-// (4H bytes for the whole kernel, served by L1) is read 8 columns at a time
-// where wh and we are on a 16-byte boundary, else column by column.
+// (4H bytes for the whole kernel, served by L1) is read 8 columns at a time;
+// SHIFT (rows whose body vectors are not on 16-byte boundaries of wh and we:
+// odd H, or tensors past a 16-byte boundary) reads it from the two aligned
+// 16-byte chunks that cover each vector (wvec_at) instead of column by column.
+// (The kernel without SHIFT is kept apart: the extra code, never run when
+// every row is aligned, made the aligned case slower.)
 //
 // The backward adds c * x_j * k_j into the CTA's partial row (row c of
 // w_partial belongs to CTA c alone and is updated in token order, so it is
@@ -138,6 +140,7 @@ __device__ __forceinline__ int row_head(const void *row, int H)
 
 // Block sums of one token's statistics in a fixed order (warp shuffles, then
 // the warps' partials in warp order).  Every thread gets the totals.
+template <int NT>
 __device__ __forceinline__ void gen_block_reduce(float px, float pk, float pg, double pa,
                                                  float4 *red, double *redd, float4 &r, double &A)
 {
@@ -153,8 +156,8 @@ __device__ __forceinline__ void gen_block_reduce(float px, float pk, float pg, d
     __syncthreads();
     r = make_float4(0.f, 0.f, 0.f, 0.f);
     A = 0.0;
-    const int nwarps = blockDim.x >> 5;
-    for (int w = 0; w < nwarps; ++w) {
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
         const float4 t = red[w];
         r.x += t.x;
         r.y += t.y;
@@ -166,57 +169,24 @@ __device__ __forceinline__ void gen_block_reduce(float px, float pk, float pg, d
 
 // Visit the columns of one row: f(j, false) for the single column j, or
 // f(j, true) for the 8 columns j..j+7 of a 16-byte vector.  Thread tid takes
-// head and tail column tid and body vectors tid, tid + blockDim.x, ...
-template <bool VEC, typename F>
+// head and tail column tid and body vectors tid, tid + NT, ... (NT threads)
+template <bool VEC, int NT, typename F>
 __device__ __forceinline__ void for_columns(const void *row, int H, F &&f)
 {
     if (!VEC) {
-        for (int j = threadIdx.x; j < H; j += blockDim.x) f(j, false);
+        for (int j = threadIdx.x; j < H; j += NT) f(j, false);
         return;
     }
     const int head = row_head(row, H);
     const int nvec = (H - head) >> 3;
     const int tail = head + 8 * nvec;
     if ((int)threadIdx.x < head) f((int)threadIdx.x, false);
-    for (int i = threadIdx.x; i < nvec; i += blockDim.x) f(head + 8 * i, true);
+    for (int i = threadIdx.x; i < nvec; i += NT) f(head + 8 * i, true);
     if (tail + (int)threadIdx.x < H) f(tail + (int)threadIdx.x, false);
 }
 
-// The same visit with the body vectors in batches of kGenBatch per thread:
-// load(b, j) for the batch's vectors (b = 0..kGenBatch-1, column j) first, so
-// that all of their loads are in flight together, then use(b, j) for each in
-// order (the order in which for_columns would visit them).  col(j) handles a
-// single column (head, tail, or every column without VEC).
-#ifndef ENGRAM_GEN_BATCH
-#define ENGRAM_GEN_BATCH 1
-#endif
-constexpr int kGenBatch = ENGRAM_GEN_BATCH;
-
-template <bool VEC, typename FC, typename FL, typename FU>
-__device__ __forceinline__ void for_columns_batched(const void *row, int H, FC &&col, FL &&load, FU &&use)
-{
-    if (!VEC) {
-        for (int j = threadIdx.x; j < H; j += blockDim.x) col(j);
-        return;
-    }
-    const int head = row_head(row, H);
-    const int nvec = (H - head) >> 3;
-    const int tail = head + 8 * nvec;
-    if ((int)threadIdx.x < head) col((int)threadIdx.x);
-    const int nt = blockDim.x;
-    for (int i0 = threadIdx.x; i0 < nvec; i0 += kGenBatch * nt) {
-#pragma unroll
-        for (int b = 0; b < kGenBatch; ++b)
-            if (i0 + b * nt < nvec) load(b, head + 8 * (i0 + b * nt));
-#pragma unroll
-        for (int b = 0; b < kGenBatch; ++b)
-            if (i0 + b * nt < nvec) use(b, head + 8 * (i0 + b * nt));
-    }
-    if (tail + (int)threadIdx.x < H) col(tail + (int)threadIdx.x);
-}
-
-template <bool VEC>
-__global__ void __launch_bounds__(kGenThreads)
+template <bool VEC, bool SHIFT, int NT>
+__global__ void __launch_bounds__(NT)
 gate_generic_fwd_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ k,
                         const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ wh,
                         const __nv_bfloat16 *__restrict__ we, int64_t T, int H, float eps,
@@ -231,25 +201,14 @@ gate_generic_fwd_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16
         __nv_bfloat16 *orow = out + t * H;
         float px = 0.f, pk = 0.f;
         double pa = 0.0;
-        uint4 xq[kGenBatch], kq[kGenBatch];
-        for_columns_batched<VEC>(
-            xr, H,
-            [&](int j) {
-                const float xv = bf(xr + j), kv = bf(kr + j);
-                px = fmaf(xv, xv, px);
-                pk = fmaf(kv, kv, pk);
-                pa = fma((double)(xv * kv), (double)wcol(wh, we, j), pa);
-            },
-            [&](int b, int j) {
-                xq[b] = *reinterpret_cast<const uint4 *>(xr + j);
-                kq[b] = *reinterpret_cast<const uint4 *>(kr + j);
-            },
-            [&](int b, int j) {
+        for_columns<VEC, NT>(xr, H, [&](int j, bool vec) {
+            if (vec) {
                 float2 xf[4], kf[4];
                 float w[8];
-                unpack4x2(xq[b], xf);
-                unpack4x2(kq[b], kf);
-                wvec_at(wh, we, j, H, w_aligned, w);
+                unpack4x2(*reinterpret_cast<const uint4 *>(xr + j), xf);
+                unpack4x2(*reinterpret_cast<const uint4 *>(kr + j), kf);
+                if (SHIFT) wvec_at(wh, we, j, H, w_aligned, w);
+                else wvec(wh, we, j, w);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     px = fmaf(xf[e].x, xf[e].x, fmaf(xf[e].y, xf[e].y, px));
@@ -257,34 +216,36 @@ gate_generic_fwd_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16
                     pa = fma((double)(xf[e].x * kf[e].x), (double)w[2 * e], pa);
                     pa = fma((double)(xf[e].y * kf[e].y), (double)w[2 * e + 1], pa);
                 }
-            });
+            } else {
+                const float xv = bf(xr + j), kv = bf(kr + j);
+                px = fmaf(xv, xv, px);
+                pk = fmaf(kv, kv, pk);
+                pa = fma((double)(xv * kv), (double)wcol(wh, we, j), pa);
+            }
+        });
         float4 r;
         double A;
-        gen_block_reduce(px, pk, 0.f, pa, red, redd, r, A);
+        gen_block_reduce<NT>(px, pk, 0.f, pa, red, redd, r, A);
         const GateScalars c = gate_scalars(r.x, r.y, A, inv_h, eps, scalar);
-        uint4 vq[kGenBatch];
-        for_columns_batched<VEC>(
-            xr, H,
-            [&](int j) { orow[j] = __float2bfloat16_rn(fmaf(c.gate, bf(vr + j), bf(xr + j))); },
-            [&](int b, int j) {
-                xq[b] = *reinterpret_cast<const uint4 *>(xr + j);
-                vq[b] = *reinterpret_cast<const uint4 *>(vr + j);
-            },
-            [&](int b, int j) {
+        for_columns<VEC, NT>(xr, H, [&](int j, bool vec) {
+            if (vec) {
                 float2 xf[4], vf[4], of[4];
-                unpack4x2(xq[b], xf);
-                unpack4x2(vq[b], vf);
+                unpack4x2(*reinterpret_cast<const uint4 *>(xr + j), xf);
+                unpack4x2(*reinterpret_cast<const uint4 *>(vr + j), vf);
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     of[e] = make_float2(fmaf(c.gate, vf[e].x, xf[e].x), fmaf(c.gate, vf[e].y, xf[e].y));
                 __stcs(reinterpret_cast<uint4 *>(orow + j), pack4x2(of));
-            });
+            } else {
+                orow[j] = __float2bfloat16_rn(fmaf(c.gate, bf(vr + j), bf(xr + j)));
+            }
+        });
         if (threadIdx.x == 0 && gate != nullptr) gate[t] = c.gate;
     }
 }
 
-template <bool VEC>
-__global__ void __launch_bounds__(kGenThreads)
+template <bool VEC, bool SHIFT, int NT>
+__global__ void __launch_bounds__(NT)
 gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloat16 *__restrict__ x,
                         const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
                         const __nv_bfloat16 *__restrict__ wh, const __nv_bfloat16 *__restrict__ we,
@@ -304,37 +265,23 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
     // array.  Every row of the CTA has that phase when G * H is a multiple of
     // 8 (odd H with the recommended G); rows of other phases take the
     // element-wise path below.
-    const int pad = VEC ? (8 - row_head(x + (int64_t)blockIdx.x * H, H)) & 7 : 0;
+    const int pad = SHIFT ? (8 - row_head(x + (int64_t)blockIdx.x * H, H)) & 7 : 0;
     float *acc = H <= kGenSmemPartial ? s_part + pad : prow;
-    for (int j = threadIdx.x; j < H; j += blockDim.x) acc[j] = 0.f;
+    for (int j = threadIdx.x; j < H; j += NT) acc[j] = 0.f;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         const __nv_bfloat16 *gr = gout + t * H, *xr = x + t * H, *kr = k + t * H, *vr = v + t * H;
         float px = 0.f, pk = 0.f, pg = 0.f;
         double pa = 0.0;
-        uint4 gq[kGenBatch], xq[kGenBatch], kq[kGenBatch], vq[kGenBatch];
-        for_columns_batched<VEC>(
-            xr, H,
-            [&](int j) {
-                const float xv = bf(xr + j), kv = bf(kr + j);
-                px = fmaf(xv, xv, px);
-                pk = fmaf(kv, kv, pk);
-                pg = fmaf(bf(gr + j), bf(vr + j), pg);
-                pa = fma((double)(xv * kv), (double)wcol(wh, we, j), pa);
-            },
-            [&](int b, int j) {
-                gq[b] = *reinterpret_cast<const uint4 *>(gr + j);
-                xq[b] = *reinterpret_cast<const uint4 *>(xr + j);
-                kq[b] = *reinterpret_cast<const uint4 *>(kr + j);
-                vq[b] = *reinterpret_cast<const uint4 *>(vr + j);
-            },
-            [&](int b, int j) {
+        for_columns<VEC, NT>(xr, H, [&](int j, bool vec) {
+            if (vec) {
                 float2 gf[4], xf[4], kf[4], vf[4];
                 float w[8];
-                unpack4x2(gq[b], gf);
-                unpack4x2(xq[b], xf);
-                unpack4x2(kq[b], kf);
-                unpack4x2(vq[b], vf);
-                wvec_at(wh, we, j, H, w_aligned, w);
+                unpack4x2(*reinterpret_cast<const uint4 *>(gr + j), gf);
+                unpack4x2(*reinterpret_cast<const uint4 *>(xr + j), xf);
+                unpack4x2(*reinterpret_cast<const uint4 *>(kr + j), kf);
+                unpack4x2(*reinterpret_cast<const uint4 *>(vr + j), vf);
+                if (SHIFT) wvec_at(wh, we, j, H, w_aligned, w);
+                else wvec(wh, we, j, w);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     px = fmaf(xf[e].x, xf[e].x, fmaf(xf[e].y, xf[e].y, px));
@@ -343,10 +290,17 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
                     pa = fma((double)(xf[e].x * kf[e].x), (double)w[2 * e], pa);
                     pa = fma((double)(xf[e].y * kf[e].y), (double)w[2 * e + 1], pa);
                 }
-            });
+            } else {
+                const float xv = bf(xr + j), kv = bf(kr + j);
+                px = fmaf(xv, xv, px);
+                pk = fmaf(kv, kv, pk);
+                pg = fmaf(bf(gr + j), bf(vr + j), pg);
+                pa = fma((double)(xv * kv), (double)wcol(wh, we, j), pa);
+            }
+        });
         float4 r;
         double A;
-        gen_block_reduce(px, pk, pg, pa, red, redd, r, A);
+        gen_block_reduce<NT>(px, pk, pg, pa, red, redd, r, A);
         const float Sg = r.z;
         const GateScalars c = gate_scalars(r.x, r.y, A, inv_h, eps, scalar);
         // chain rule through sigmoid, signed_sqrt (|s| clamped at 1e-6), scalar
@@ -356,28 +310,15 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
         const float c2 = dd * c.d * c.rx * c.rx * inv_h;
         const float c3 = dd * c.d * c.rk * c.rk * inv_h;
         __nv_bfloat16 *dxr = dx + t * H, *dkr = dk + t * H, *dvr = dv + t * H;
-        for_columns_batched<VEC>(
-            xr, H,
-            [&](int j) {
-                const float gv = bf(gr + j), xv = bf(xr + j), kv = bf(kr + j);
-                const float cw = c1 * wcol(wh, we, j);
-                dxr[j] = __float2bfloat16_rn(fmaf(-c2, xv, fmaf(cw, kv, gv)));
-                dkr[j] = __float2bfloat16_rn(fmaf(-c3, kv, cw * xv));
-                dvr[j] = __float2bfloat16_rn(c.gate * gv);
-                acc[j] = fmaf(c1, xv * kv, acc[j]);
-            },
-            [&](int bb, int j) {
-                gq[bb] = *reinterpret_cast<const uint4 *>(gr + j);
-                xq[bb] = *reinterpret_cast<const uint4 *>(xr + j);
-                kq[bb] = *reinterpret_cast<const uint4 *>(kr + j);
-            },
-            [&](int bb, int j) {
+        for_columns<VEC, NT>(xr, H, [&](int j, bool vec) {
+            if (vec) {
                 float2 gf[4], xf[4], kf[4], a[4], b[4], cv[4];
                 float w[8], pr[8];
-                unpack4x2(gq[bb], gf);
-                unpack4x2(xq[bb], xf);
-                unpack4x2(kq[bb], kf);
-                wvec_at(wh, we, j, H, w_aligned, w);
+                unpack4x2(*reinterpret_cast<const uint4 *>(gr + j), gf);
+                unpack4x2(*reinterpret_cast<const uint4 *>(xr + j), xf);
+                unpack4x2(*reinterpret_cast<const uint4 *>(kr + j), kf);
+                if (SHIFT) wvec_at(wh, we, j, H, w_aligned, w);
+                else wvec(wh, we, j, w);
                 const bool acc4 = (reinterpret_cast<uintptr_t>(acc + j) & 15u) == 0;
                 if (acc4) {
                     const float4 p0 = *reinterpret_cast<const float4 *>(acc + j);
@@ -408,11 +349,19 @@ gate_generic_bwd_kernel(const __nv_bfloat16 *__restrict__ gout, const __nv_bfloa
                 __stcs(reinterpret_cast<uint4 *>(dxr + j), pack4x2(a));
                 __stcs(reinterpret_cast<uint4 *>(dkr + j), pack4x2(b));
                 __stcs(reinterpret_cast<uint4 *>(dvr + j), pack4x2(cv));
-            });
+            } else {
+                const float gv = bf(gr + j), xv = bf(xr + j), kv = bf(kr + j);
+                const float cw = c1 * wcol(wh, we, j);
+                dxr[j] = __float2bfloat16_rn(fmaf(-c2, xv, fmaf(cw, kv, gv)));
+                dkr[j] = __float2bfloat16_rn(fmaf(-c3, kv, cw * xv));
+                dvr[j] = __float2bfloat16_rn(c.gate * gv);
+                acc[j] = fmaf(c1, xv * kv, acc[j]);
+            }
+        });
     }
     if (acc != prow) {
         __syncthreads();
-        for (int j = threadIdx.x; j < H; j += blockDim.x) prow[j] = acc[j];
+        for (int j = threadIdx.x; j < H; j += NT) prow[j] = acc[j];
     }
 }
 

@@ -525,14 +525,12 @@ gate_bwd_kernel(const uint4 *__restrict__ gout, const uint4 *__restrict__ x,
             rbd[warp] = pa;
         }
         if (__syncthreads_or(!ok)) {
+            // (with the fused reduction the CTA then takes no ticket: the
+            // CTAs waiting in the tail give up at their own time limit)
             if (tid == 0) {
                 record_device_error(kErrPipelineTimeout);
                 gate_drain(bar0, i, nrows, nstage);
             }
-            // With the fused reduction: give up on the remaining tokens but
-            // still take part in the tail below, so that its tickets stay
-            // consistent.
-            if (FUSED) break;
             return;
         }
         if (tid == 0 && i + nstage < nrows)
