@@ -151,9 +151,10 @@ gbwd_mark_kernel(const int64_t *__restrict__ idx, const __grid_constant__ Gather
 // (lane l: the round's entry l); a round's unique entries are dealt to the
 // warp's 32 / LPR groups of LPR lanes, U at a time per group, lane cv owning
 // the columns [8 cv, 8 cv + 8).  The kernel releases its dependents as soon
-// as it starts, and its grid leaves one CTA slot per SM free, so that the
-// staging and list kernels launched after it run beside it.  Up to four CTAs
-// per SM fit (64 registers a thread, a few spilled).
+// as it starts, so that the staging kernel launched after it is scheduled as
+// its CTAs leave.  Four CTAs per SM at 64 registers; U = 2 rows in flight
+// per group (no spills) beat U = 4 (a few registers spilled): 194 against
+// 201 us per call at the full-path workload, same bits.
 template <int LPR, int U>
 __global__ void __launch_bounds__(kUniqThreads, 4)
 gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_rows,
@@ -522,8 +523,9 @@ __device__ __forceinline__ void add_bf16x8(double a[8], const uint4 &q)
 // from those registers; a row read several times is summed afterwards (a long
 // run of one hot row by the whole warp, the groups splitting its gradients),
 // so the fp64 accumulators of that case do not add to the registers of the
-// common one.  Four CTAs per SM (64 registers a thread, a few spilled) run
-// faster than three (209 -> 206 us per call at the full-path workload).
+// common one.  Four CTAs per SM (64 registers a thread) run faster than
+// three (209 -> 206 us per call at the full-path workload), and one segment
+// at a time per group (U = 1) faster than two (194 -> 191 us).
 template <int LPR, int U>
 __global__ void __launch_bounds__(kSegThreads, 4)
 gbwd_segment_kernel(const uint32_t *__restrict__ keys, const uint32_t *__restrict__ vals,

@@ -164,13 +164,13 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
         const unsigned ut = (unsigned)engram::kUniqThreads;
         const uint32_t *dm = dupmap;
         if (nv <= 4)
-            e = launch_pdl(engram::gbwd_unique_kernel<4, 4>, ub, ut, s, idx, rows, p, dm, tab4);
+            e = launch_pdl(engram::gbwd_unique_kernel<4, 2>, ub, ut, s, idx, rows, p, dm, tab4);
         else if (nv <= 8)
-            e = launch_pdl(engram::gbwd_unique_kernel<8, 4>, ub, ut, s, idx, rows, p, dm, tab4);
+            e = launch_pdl(engram::gbwd_unique_kernel<8, 2>, ub, ut, s, idx, rows, p, dm, tab4);
         else if (nv <= 16)
-            e = launch_pdl(engram::gbwd_unique_kernel<16, 4>, ub, ut, s, idx, rows, p, dm, tab4);
+            e = launch_pdl(engram::gbwd_unique_kernel<16, 2>, ub, ut, s, idx, rows, p, dm, tab4);
         else
-            e = launch_pdl(engram::gbwd_unique_kernel<32, 4>, ub, ut, s, idx, rows, p, dm, tab4);
+            e = launch_pdl(engram::gbwd_unique_kernel<32, 2>, ub, ut, s, idx, rows, p, dm, tab4);
     }
     // 3. the entries of rows read more than once, staged per tile (into the
     //    second buffer pair) with the first radix pass's tile histograms
@@ -209,16 +209,16 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     const uint32_t *kc = keys[cur], *vc = vals[cur];
     if (e == cudaSuccess) {
         if (nv <= 4)
-            e = launch_pdl(engram::gbwd_segment_kernel<4, 2>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
+            e = launch_pdl(engram::gbwd_segment_kernel<4, 1>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
         else if (nv <= 8)
-            e = launch_pdl(engram::gbwd_segment_kernel<8, 2>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
+            e = launch_pdl(engram::gbwd_segment_kernel<8, 1>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
         else if (nv <= 16)
-            e = launch_pdl(engram::gbwd_segment_kernel<16, 2>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
+            e = launch_pdl(engram::gbwd_segment_kernel<16, 1>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
         else
-            e = launch_pdl(engram::gbwd_segment_kernel<32, 2>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
+            e = launch_pdl(engram::gbwd_segment_kernel<32, 1>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
     }
     // one warp per listed chunk (a warp loops when more than 4096 are listed);
