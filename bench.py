@@ -436,9 +436,9 @@ def run_ours(args):
         gbwd.update({"traffic": committed_traffic("gather_bwd", T), "unique_rows": uniq,
                      "entries": T * L * J, "launches": GATHER_BWD_LAUNCHES,
                      "what": "engram_gather_bwd on the step's indices: rows read once updated "
-                             "in place, the rest listed, radix-sorted by row and summed in fp64; "
-                             "fp32 table-gradient update; 20 calls back to back, CUDA events "
-                             "around them"})
+                             "in place, the rest listed, radix-sorted by row and summed in fp64 "
+                             "on a side stream beside the update; fp32 table-gradient update; "
+                             "20 calls back to back, CUDA events around them"})
         del d_rows, d_tables, ws
 
     kern = {n: kernel_entry(per_kernel_ms[n] * 1e3, ab[n], peak) for n in names}

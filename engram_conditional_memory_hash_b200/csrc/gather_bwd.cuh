@@ -18,10 +18,9 @@
 //      matter: a row ends up in dupmap exactly when two or more entries read it);
 //   2. unique: entries whose row is not in dupmap update their row directly
 //      with one rounding: fp32((double)d_tables[r] + g).  This is the
-//      bandwidth-bound part; it runs on a persistent grid that leaves room on
-//      every SM, and the list kernels below (stage, sort, segments) are
-//      scheduled beside it at once (they touch only rows in dupmap, it only
-//      the others);
+//      bandwidth-bound part; the list kernels below (stage, sort, segments,
+//      carries) run beside it on a stream of higher priority (they touch only
+//      rows in dupmap, it only the others);
 //      stage: each tile of entries stages the (key, e) pairs of its entries
 //      whose row is in dupmap, in position order, with their count and
 //      first-digit histogram;
@@ -66,9 +65,11 @@ constexpr int kSegChunk = 64;                           // sorted entries per wa
 constexpr int kSegThreads = 256;
 constexpr int kCarryThreads = 256;
 constexpr int kMarkThreads = 256;
-constexpr int kUniqThreads = 256;
-constexpr int kUniqWarpEntries = 128;                   // entries per warp in unique/compact
+constexpr int kUniqThreads = 256;                       // staging kernel
+constexpr int kUniqWarpEntries = 128;                   // entries per warp in unique/stage
 constexpr int kUniqTile = kUniqThreads / 32 * kUniqWarpEntries;
+constexpr int kUpdThreads = 64;                         // unique-row update
+constexpr int kUpdTile = kUpdThreads / 32 * kUniqWarpEntries;
 static_assert(kSortThreads == kRadixBins, "one thread per digit in the histogram epilogue");
 static_assert(kUniqTile == kSortTile, "the first radix pass reads the unique kernel's staged tiles");
 
@@ -146,17 +147,17 @@ gbwd_mark_kernel(const int64_t *__restrict__ idx, const __grid_constant__ Gather
 }
 
 // Rows read by one entry only: d_tables[r] = fp32((double)d_tables[r] + g).
-// Persistent: CTA b handles the tiles b, b + gridDim.x, ... of kUniqTile
-// entries; warp w of a tile handles kUniqWarpEntries entries in rounds of 32
+// CTA b handles the tiles b, b + gridDim.x, ... of kUpdTile entries (one
+// tile per CTA as launched, so that CTAs are short-lived and the list
+// kernels, on a stream of higher priority, get SM slots as they finish:
+// 64-thread CTAs measured 1.5 % faster per call than 256-thread ones);
+// warp w of a tile handles kUniqWarpEntries entries in rounds of 32
 // (lane l: the round's entry l); a round's unique entries are dealt to the
 // warp's 32 / LPR groups of LPR lanes, U at a time per group, lane cv owning
-// the columns [8 cv, 8 cv + 8).  The kernel releases its dependents as soon
-// as it starts, so that the staging kernel launched after it is scheduled as
-// its CTAs leave.  Four CTAs per SM at 64 registers; U = 2 rows in flight
-// per group (no spills) beat U = 4 (a few registers spilled): 194 against
-// 201 us per call at the full-path workload, same bits.
+// the columns [8 cv, 8 cv + 8).  32 warps per SM at 60 registers; U = 2
+// rows in flight per group (no spills) beat U = 4 (a few registers spilled).
 template <int LPR, int U>
-__global__ void __launch_bounds__(kUniqThreads, 4)
+__global__ void __launch_bounds__(kUpdThreads, 1024 / kUpdThreads)
 gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_rows,
                    const __grid_constant__ GatherBwdParams p, const uint32_t *__restrict__ dupmap,
                    float4 *__restrict__ d_tables)
@@ -168,9 +169,9 @@ gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_
     const int nv = p.D >> 3;
     const bool col = cv < nv;
     pdl_wait_and_release();
-    const int64_t ntiles = (p.N + kUniqTile - 1) / kUniqTile;
+    const int64_t ntiles = (p.N + kUpdTile - 1) / kUpdTile;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int64_t base = tile * kUniqTile + (int64_t)warp * kUniqWarpEntries;
+        const int64_t base = tile * kUpdTile + (int64_t)warp * kUniqWarpEntries;
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
             const int64_t e = base + r * 32 + lane;
@@ -219,9 +220,8 @@ gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_
 // histogram of their lowest 8 key bits to hist[digit * ntiles + t] (the first
 // radix pass reads the staged tiles directly), and adds the count to *m_out,
 // the length of the list.
-// Launched right after the unique-row update and run beside it: it does not
-// wait for that kernel (which it does not depend on) and reads dupmap, which
-// the mark kernel wrote before the update kernel started, through L2.
+// It runs beside the unique-row update (on another stream), after the mark
+// kernel; it reads dupmap through L2.
 __global__ void __launch_bounds__(kUniqThreads)
 gbwd_stage_kernel(const int64_t *__restrict__ idx, const __grid_constant__ GatherBwdParams p,
                   const uint32_t *__restrict__ dupmap, uint32_t *__restrict__ stage_keys,

@@ -7,15 +7,6 @@ namespace {
 
 constexpr int64_t kGbwdMaxEntries = int64_t(1) << 30;
 
-// CTAs per SM of the persistent unique-row update: as many as fit (four).
-// Leaving a slot free for the staging and list kernels launched after it was
-// measured slower (217 us per call with three, 237 with two, 198 with four at
-// the full-path workload): the update needs every warp it can get.
-#ifndef ENGRAM_GBWD_UNIQ_PER_SM
-#define ENGRAM_GBWD_UNIQ_PER_SM 4
-#endif
-constexpr int kGbwdUniqPerSm = ENGRAM_GBWD_UNIQ_PER_SM;
-
 // Offsets (bytes, 256-aligned) of the gather backward's scratch in the
 // caller's workspace.  A region zeroed by every call first: the `seen` and
 // `dupmap` bitmaps (one bit per table row) and the counters (list length,
@@ -61,6 +52,38 @@ GbwdLayout gbwd_layout(int64_t N, int D, int64_t R)
     g.carry_list = take((size_t)g.nchunks * 4);
     g.total = N > 0 ? off : 0;
     return g;
+}
+
+// The list kernels (stage, sort, segments, carries) touch only the rows read
+// more than once and the unique-row update only the others, so they run side
+// by side: the list kernels on a side stream of the highest priority, forked
+// from and joined back into the caller's stream with two events.  With the
+// priority the list kernels' CTAs take the SM slots the update's short-lived
+// CTAs free, ahead of the update's remaining CTAs.  One side stream and the
+// two events per device, created on first use and kept until the process
+// exits; the mutex is held while a call enqueues its work (the events are
+// shared), so calls from several host threads take turns on the side stream.
+struct GbwdFork {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_gbwd_mutex;
+GbwdFork g_gbwd_fork[kMaxDevices];
+
+// With g_gbwd_mutex held.
+engram_status_t gbwd_fork_objects(int dev, GbwdFork **out)
+{
+    GbwdFork &f = g_gbwd_fork[dev];
+    if (f.side == nullptr) {
+        int least = 0, greatest = 0;
+        cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&f.side, cudaStreamNonBlocking, greatest);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&f.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&f.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) return cuda_fail(e, "gather_bwd side stream");
+    }
+    *out = &f;
+    return ENGRAM_OK;
 }
 
 engram_status_t check_gbwd_sizes(int64_t T, int32_t L, int32_t J, int32_t D)
@@ -157,26 +180,37 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
         e = launch_pdl(engram::gbwd_mark_kernel, mblocks, (unsigned)engram::kMarkThreads, s, idx, p, seen,
                        dupmap);
     }
-    // 2. rows read once: update in place, on a persistent grid that leaves a
-    //    CTA slot free on every SM; the kernels from 3 on run beside it
-    if (e == cudaSuccess) {
-        const unsigned ub = (unsigned)std::min<int64_t>(g.utiles, (int64_t)dev.sms * kGbwdUniqPerSm);
-        const unsigned ut = (unsigned)engram::kUniqThreads;
+    // 2. fork: the list kernels (3-5) on the side stream, the unique-row
+    //    update on the caller's stream, joined at the end
+    std::lock_guard<std::mutex> fork_lock(g_gbwd_mutex);
+    GbwdFork *fk = nullptr;
+    if (e == cudaSuccess && (st = gbwd_fork_objects(dev.ordinal, &fk)) != ENGRAM_OK) return st;
+    if (e == cudaSuccess) e = cudaEventRecord(fk->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(fk->side, fk->fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "gather_bwd fork");
+    cudaStream_t ls = fk->side;
+    // the rows read once: updated in place on the caller's stream, one CTA per
+    // tile of entries (short-lived CTAs, so that the list kernels find slots)
+    {
+        const unsigned ub = (unsigned)((N + engram::kUpdTile - 1) / engram::kUpdTile);
+        const unsigned ut = (unsigned)engram::kUpdThreads;
         const uint32_t *dm = dupmap;
-        if (nv <= 4)
-            e = launch_pdl(engram::gbwd_unique_kernel<4, 2>, ub, ut, s, idx, rows, p, dm, tab4);
-        else if (nv <= 8)
-            e = launch_pdl(engram::gbwd_unique_kernel<8, 2>, ub, ut, s, idx, rows, p, dm, tab4);
-        else if (nv <= 16)
-            e = launch_pdl(engram::gbwd_unique_kernel<16, 2>, ub, ut, s, idx, rows, p, dm, tab4);
-        else
-            e = launch_pdl(engram::gbwd_unique_kernel<32, 2>, ub, ut, s, idx, rows, p, dm, tab4);
+        auto uniq = [&](auto kern) {
+            kern<<<ub, ut, 0, s>>>(idx, rows, p, dm, tab4);
+            return cudaGetLastError();
+        };
+        e = nv <= 4 ? uniq(engram::gbwd_unique_kernel<4, 2>)
+          : nv <= 8 ? uniq(engram::gbwd_unique_kernel<8, 2>)
+          : nv <= 16 ? uniq(engram::gbwd_unique_kernel<16, 2>)
+                     : uniq(engram::gbwd_unique_kernel<32, 2>);
     }
     // 3. the entries of rows read more than once, staged per tile (into the
     //    second buffer pair) with the first radix pass's tile histograms
-    if (e == cudaSuccess)
-        e = launch_pdl(engram::gbwd_stage_kernel, (unsigned)g.utiles, (unsigned)engram::kUniqThreads, s, idx,
-                       p, static_cast<const uint32_t *>(dupmap), keys[1], vals[1], tile_cnt, hist, m_dev);
+    if (e == cudaSuccess) {
+        engram::gbwd_stage_kernel<<<(unsigned)g.utiles, (unsigned)engram::kUniqThreads, 0, ls>>>(
+            idx, p, static_cast<const uint32_t *>(dupmap), keys[1], vals[1], tile_cnt, hist, m_dev);
+        e = cudaGetLastError();
+    }
     // 4. stable radix sort by row of the staged entries into a contiguous
     //    list; keys lie in [0, R): sort on the bit length of R - 1
     int nbits = 0;
@@ -188,14 +222,14 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     for (int pass = 0; pass < npasses && e == cudaSuccess; ++pass) {
         const int shift = 8 * pass;
         if (pass > 0)
-            e = launch_pdl(engram::gbwd_hist_kernel, stiles, T_, s, static_cast<const uint32_t *>(keys[cur]),
+            e = launch_pdl(engram::gbwd_hist_kernel, stiles, T_, ls, static_cast<const uint32_t *>(keys[cur]),
                            m_c, shift, hist);
         if (e == cudaSuccess)
             e = launch_pdl(engram::gbwd_digit_scan_kernel, (unsigned)engram::kRadixBins,
-                           (unsigned)engram::kScanThreads, s, hist, m_c, pass == 0 ? g.utiles : int64_t(0),
+                           (unsigned)engram::kScanThreads, ls, hist, m_c, pass == 0 ? g.utiles : int64_t(0),
                            totals);
         if (e == cudaSuccess)
-            e = launch_pdl(engram::gbwd_scatter_kernel, pass == 0 ? (unsigned)g.utiles : stiles, T_, s,
+            e = launch_pdl(engram::gbwd_scatter_kernel, pass == 0 ? (unsigned)g.utiles : stiles, T_, ls,
                            static_cast<const uint32_t *>(keys[cur]), static_cast<const uint32_t *>(vals[cur]),
                            m_c, pass == 0 ? static_cast<const uint32_t *>(tile_cnt) : no_cnt, shift,
                            static_cast<const uint32_t *>(hist), static_cast<const uint32_t *>(totals),
@@ -209,22 +243,19 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     const uint32_t *kc = keys[cur], *vc = vals[cur];
     if (e == cudaSuccess) {
         if (nv <= 4)
-            e = launch_pdl(engram::gbwd_segment_kernel<4, 1>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
+            e = launch_pdl(engram::gbwd_segment_kernel<4, 1>, blocks, S_, ls, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
         else if (nv <= 8)
-            e = launch_pdl(engram::gbwd_segment_kernel<8, 1>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
+            e = launch_pdl(engram::gbwd_segment_kernel<8, 1>, blocks, S_, ls, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
         else if (nv <= 16)
-            e = launch_pdl(engram::gbwd_segment_kernel<16, 1>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
+            e = launch_pdl(engram::gbwd_segment_kernel<16, 1>, blocks, S_, ls, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
         else
-            e = launch_pdl(engram::gbwd_segment_kernel<32, 1>, blocks, S_, s, kc, vc, rows, p, tab4, carry_a,
+            e = launch_pdl(engram::gbwd_segment_kernel<32, 1>, blocks, S_, ls, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
     }
-    // one warp per listed chunk (a warp loops when more than 4096 are listed);
-    // launched without the programmatic dependency, so that it starts only
-    // when everything before it in the stream (the unique-row update included)
-    // has completed, and the call's last kernel ends after all of its work
+    // one warp per listed chunk (a warp loops when more than 4096 are listed)
     const int64_t carry_warps = std::min<int64_t>(g.nchunks, 4096);
     const unsigned carry_blocks = (unsigned)((carry_warps + engram::kCarryThreads / 32 - 1) /
                                              (engram::kCarryThreads / 32));
@@ -232,15 +263,18 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     const double *ca = carry_a, *cb = carry_b;
     const uint32_t *cl = carry_list, *cn = carry_count;
     if (e == cudaSuccess) {
-        auto carry = [&](auto kern) {
-            kern<<<carry_blocks, CT, 0, s>>>(kc, p, d_tables, ca, cb, cl, cn);
-            return cudaGetLastError();
-        };
+        auto carry = [&](auto kern) { return launch_pdl(kern, carry_blocks, CT, ls, kc, p, d_tables, ca, cb, cl, cn); };
         e = D <= 32 ? carry(engram::gbwd_carry_kernel<1>)
           : D <= 64 ? carry(engram::gbwd_carry_kernel<2>)
           : D <= 128 ? carry(engram::gbwd_carry_kernel<4>)
                      : carry(engram::gbwd_carry_kernel<8>);
     }
+    // join: the caller's stream continues once the list kernels are done
+    // (recorded even after a failed launch, so that the side stream never
+    // runs ahead of a later call's fork)
+    const cudaError_t ej = cudaEventRecord(fk->join, ls);
+    const cudaError_t ew = ej == cudaSuccess ? cudaStreamWaitEvent(s, fk->join, 0) : ej;
+    if (e == cudaSuccess) e = ew;
     if (e != cudaSuccess) return cuda_fail(e, "gather_bwd launch");
     return ENGRAM_OK;
 }

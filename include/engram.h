@@ -15,7 +15,9 @@
  * Conventions shared by every call:
  *   - Device pointers point to CUDA device memory of the current device.  The
  *     caller allocates every buffer and keeps ownership; the library allocates
- *     nothing and keeps no state between calls.
+ *     no device memory.  Per device it keeps, from the first call that needs
+ *     them until the process exits, host-side launch settings of the gate
+ *     calls and, for engram_gather_bwd, one stream and two events.
  *   - Every compute call is asynchronous on `stream` (NULL: the legacy default
  *     stream) and never synchronises.  Outputs are valid once the stream has
  *     reached the call.
@@ -160,6 +162,16 @@ ENGRAM_API int64_t engram_gather_bwd_workspace_size(int64_t T, int32_t L, int32_
  *             aligned, owned by the caller; its contents need not be
  *             initialised and are meaningless afterwards.  Calls in flight at
  *             the same time need separate workspaces.
+ *
+ * Streams: the kernels for the rows read more than once run on a stream of
+ * the device's highest priority that the library creates on the first call
+ * (one per device), forked from `stream` and joined back into it with two
+ * events, so the call is ordered on `stream` like any other.  Calls from
+ * several host threads take turns while they enqueue, and their side work
+ * runs in the order they enqueued.  A call may be captured into a CUDA graph
+ * once an earlier call has created the side stream; until that capture ends,
+ * the side stream belongs to it, so no other thread may call
+ * engram_gather_bwd on the same device meanwhile.
  */
 ENGRAM_API engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int32_t J,
                                   const int64_t *table_sizes, const void *d_rows, int32_t D,

@@ -264,3 +264,112 @@ def test_full_path_size_sampled(oracle_lib):
     absum = np.abs(_widen(d_rows)).reshape(-1, w.D).sum(0)
     # each row value carries one fp32 rounding (2^-24 relative)
     assert np.all(np.abs(colsum.cpu().numpy() - want_sum) <= 2.0 ** -23 * absum)
+
+
+def _side_stream_cases(n):
+    """n independent (idx, table sizes, d_rows) problems with many repeated rows,
+    so that every call has work on the library's side stream."""
+    cases = []
+    for k in range(n):
+        r = np.random.default_rng(100 + k)
+        sizes = np.full((2, 4), 300 + 50 * k, dtype=np.int64)
+        T = 20000 + 3000 * k
+        idx = r.integers(0, int(sizes[0, 0]), size=(T, 2, 4), dtype=np.int64)
+        d_rows = inputs.f32_to_bf16_bits(r.standard_normal((T, 2, 4, 32)).astype(np.float32))
+        cases.append((torch.from_numpy(idx).cuda(), sizes, to_dev_bf16(d_rows)))
+    return cases
+
+
+def _serial(cases, repeats):
+    out = []
+    for idx, sizes, d_rows in cases:
+        t = torch.zeros((int(sizes.sum()), 32), dtype=torch.float32, device="cuda")
+        for _ in range(repeats):
+            eng.engram_gather_bwd(idx, sizes, d_rows, t)
+        out.append(t)
+    torch.cuda.synchronize()
+    return out
+
+
+def _workspaces(cases):
+    return [torch.empty(eng.engram_gather_bwd_workspace_size(idx.shape[0], 2, 4, 32, int(sizes.sum())),
+                        dtype=torch.uint8, device="cuda") for idx, sizes, _ in cases]
+
+
+def _bits_equal(a, b):
+    return torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
+def test_side_stream_calls_on_two_streams():
+    # calls on two caller streams, interleaved: the library's side stream is
+    # shared, each call joins back into its own stream; results as if serial
+    cases = _side_stream_cases(2)
+    want = _serial(cases, 3)
+    ws = _workspaces(cases)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    got = [torch.zeros_like(w) for w in want]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for (idx, sizes, d_rows), t, w, s in zip(cases, got, ws, streams):
+            eng.engram_gather_bwd(idx, sizes, d_rows, t, workspace=w, stream=s)
+    # what follows on each caller stream sees the finished result
+    sums = []
+    for t, s in zip(got, streams):
+        with torch.cuda.stream(s):
+            sums.append(t.double().sum())
+    torch.cuda.synchronize()
+    assert eng.engram_read_device_error() == 0
+    for g, w, sm in zip(got, want, sums):
+        assert _bits_equal(g, w)
+        assert sm.item() == w.double().sum().item()
+
+
+def test_side_stream_calls_from_two_threads():
+    import threading
+
+    cases = _side_stream_cases(2)
+    want = _serial(cases, 4)
+    ws = _workspaces(cases)
+    got = [torch.zeros_like(w) for w in want]
+    torch.cuda.synchronize()
+    errors = []
+
+    def worker(k):
+        try:
+            s = torch.cuda.Stream()
+            idx, sizes, d_rows = cases[k]
+            for _ in range(4):
+                eng.engram_gather_bwd(idx, sizes, d_rows, got[k], workspace=ws[k], stream=s)
+            s.synchronize()
+        except Exception as exc:       # reported on the main thread
+            errors.append(exc)
+
+    th = [threading.Thread(target=worker, args=(k,)) for k in range(2)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errors, errors
+    for g, w in zip(got, want):
+        assert _bits_equal(g, w)
+
+
+def test_side_stream_in_cuda_graph():
+    # the fork and join are captured like any other stream work; the first
+    # call on the device (which creates the side stream) happens before capture
+    cases = _side_stream_cases(1)
+    idx, sizes, d_rows = cases[0]
+    want = _serial(cases, 2)[0]
+    ws = _workspaces(cases)[0]
+    t = torch.zeros_like(want)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        eng.engram_gather_bwd(idx, sizes, d_rows, t, workspace=ws)
+    torch.cuda.synchronize()
+    assert not t.any()                 # captured, not run
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert eng.engram_read_device_error() == 0
+    assert _bits_equal(t, want)
+    del g
