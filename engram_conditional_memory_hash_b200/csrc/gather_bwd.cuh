@@ -69,7 +69,8 @@ constexpr int kUniqThreads = 256;                       // staging kernel
 constexpr int kUniqWarpEntries = 128;                   // entries per warp in unique/stage
 constexpr int kUniqTile = kUniqThreads / 32 * kUniqWarpEntries;
 constexpr int kUpdThreads = 64;                         // unique-row update
-constexpr int kUpdTile = kUpdThreads / 32 * kUniqWarpEntries;
+constexpr int kUpdWarpEntries = 32;                     // entries per warp in the update
+constexpr int kUpdTile = kUpdThreads / 32 * kUpdWarpEntries;
 static_assert(kSortThreads == kRadixBins, "one thread per digit in the histogram epilogue");
 static_assert(kUniqTile == kSortTile, "the first radix pass reads the unique kernel's staged tiles");
 
@@ -150,12 +151,13 @@ gbwd_mark_kernel(const int64_t *__restrict__ idx, const __grid_constant__ Gather
 // CTA b handles the tiles b, b + gridDim.x, ... of kUpdTile entries (one
 // tile per CTA as launched, so that CTAs are short-lived and the list
 // kernels, on a stream of higher priority, get SM slots as they finish:
-// 64-thread CTAs measured 1.5 % faster per call than 256-thread ones);
-// warp w of a tile handles kUniqWarpEntries entries in rounds of 32
-// (lane l: the round's entry l); a round's unique entries are dealt to the
-// warp's 32 / LPR groups of LPR lanes, U at a time per group, lane cv owning
-// the columns [8 cv, 8 cv + 8).  32 warps per SM at 60 registers; U = 2
-// rows in flight per group (no spills) beat U = 4 (a few registers spilled).
+// per call, 64-entry CTAs of 64 threads took 157 us, 128-entry ones 166,
+// 256-entry ones 178, 1024-entry ones of 256 threads 181); warp w of a tile
+// handles kUpdWarpEntries entries in rounds of 32 (lane l: the round's entry
+// l); a round's unique entries are dealt to the warp's 32 / LPR groups of
+// LPR lanes, U at a time per group, lane cv owning the columns
+// [8 cv, 8 cv + 8).  32 warps per SM at 60 registers; U = 2 rows in flight
+// per group (157 us per call) beat U = 1 (163-168) and U = 4 (160).
 template <int LPR, int U>
 __global__ void __launch_bounds__(kUpdThreads, 1024 / kUpdThreads)
 gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_rows,
@@ -163,7 +165,7 @@ gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_
                    float4 *__restrict__ d_tables)
 {
     constexpr int GPW = 32 / LPR;
-    constexpr int RW = kUniqWarpEntries / 32;
+    constexpr int RW = kUpdWarpEntries / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int grp = lane / LPR, cv = lane % LPR;
     const int nv = p.D >> 3;
@@ -171,7 +173,7 @@ gbwd_unique_kernel(const int64_t *__restrict__ idx, const uint4 *__restrict__ d_
     pdl_wait_and_release();
     const int64_t ntiles = (p.N + kUpdTile - 1) / kUpdTile;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int64_t base = tile * kUpdTile + (int64_t)warp * kUniqWarpEntries;
+        const int64_t base = tile * kUpdTile + (int64_t)warp * kUpdWarpEntries;
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
             const int64_t e = base + r * 32 + lane;
