@@ -192,6 +192,49 @@ def test_empty_and_argument_errors():
         eng.engram_gather_bwd(idx, sizes, d_rows, d_tables, workspace=small)
 
 
+@pytest.mark.parametrize("sizes", [[100, 100], [128, 128], [128, 129], [150, 150, 100], [40000, 30000]])
+def test_sort_levels(oracle_lib, sizes):
+    # total rows R = 200, 256 (keys of 8 bits: one radix pass), 257 (9 bits:
+    # a second pass on one bit), 400, 70000 (17 bits: three passes); every row
+    # read several times
+    r = np.random.default_rng(len(sizes) + sum(sizes))
+    sizes = np.array(sizes, dtype=np.int64).reshape(1, -1)
+    T, D = 3000, 16
+    idx_np = (r.random((T,) + sizes.shape) ** 3 * sizes[None]).astype(np.int64)
+    d_rows = inputs.f32_to_bf16_bits(r.standard_normal((T,) + sizes.shape + (D,)).astype(np.float32))
+    R = int(sizes.sum())
+    init = r.standard_normal((R, D)).astype(np.float32).astype(np.float64)
+    got = _run(torch.from_numpy(idx_np).cuda(), sizes, d_rows, init)
+    want, tol, touched = _expect(oracle_lib, idx_np, sizes, d_rows, init)
+    _check(got, want, tol, touched, init)
+
+
+def test_every_token_the_same():
+    # the degenerate input: every token reads the same row of each of 16 tables
+    # of ~1M rows, so 16 rows hold all 20000 entries each: one digit value per
+    # radix pass takes nearly every entry, and each row's run spans 313 chunks
+    # (the result: each of those rows gets the column sums of its table's
+    # gradients)
+    r = np.random.default_rng(9)
+    L, J, T, D = 2, 8, 20000, 8
+    sizes = inputs.consecutive_primes(1000003, L * J).reshape(L, J)
+    pick = r.integers(0, 1000003, size=(1, L, J))
+    idx_np = np.broadcast_to(pick, (T, L, J)).astype(np.int64).copy()
+    d_rows = inputs.f32_to_bf16_bits(r.standard_normal((T, L, J, D)).astype(np.float32))
+    R = int(sizes.sum())
+    d_tables = torch.zeros((R, D), dtype=torch.float32, device="cuda")
+    eng.engram_gather_bwd(torch.from_numpy(idx_np).cuda(), sizes, to_dev_bf16(d_rows), d_tables)
+    assert eng.engram_read_device_error() == 0
+    first = np.concatenate([[0], np.cumsum(sizes.ravel())[:-1]])
+    rows = first + pick.ravel()
+    g = _widen(d_rows).reshape(T, L * J, D)
+    want = g.sum(axis=0)
+    absum = np.abs(g).sum(axis=0)
+    got = d_tables[torch.from_numpy(rows).cuda()].double().cpu().numpy()
+    assert np.all(np.abs(got - want) <= 2.0 ** -24 * np.abs(want) + 2 * T * 2.0 ** -52 * absum)
+    assert int((d_tables != 0).any(dim=1).sum()) == L * J
+
+
 def test_four_radix_passes(oracle_lib):
     # 16 tables of ~4.19M rows (67M rows in all, more than 2^24): row keys need
     # four 8-bit radix passes; a Zipf-like skew makes many rows repeat.  D = 8
