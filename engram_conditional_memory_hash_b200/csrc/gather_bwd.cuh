@@ -77,6 +77,7 @@ static_assert(kUniqTile == kSortTile, "the first radix pass reads the unique ker
 struct GatherBwdParams {
     int64_t N;                          // entries: T * L * J
     int32_t LJ;                         // tables
+    uint64_t lj_inv;                    // floor(2^64 / LJ) + 1 (LJ > 1): e / LJ = umulhi(e, lj_inv), e < 2^32
     int32_t D;                          // row width in bf16 values (even)
     uint32_t R;                         // rows of all tables
     uint32_t P[kHashMaxTables];         // rows of table q
@@ -87,7 +88,8 @@ struct GatherBwdParams {
 __device__ __forceinline__ uint32_t gbwd_key(const int64_t *__restrict__ idx, int64_t e,
                                              const GatherBwdParams &p, bool record)
 {
-    const int q = (int)((uint32_t)e % (uint32_t)p.LJ);
+    const uint32_t e32 = (uint32_t)e;   // entries < 2^30
+    const int q = p.LJ == 1 ? 0 : (int)(e32 - (uint32_t)__umul64hi((uint64_t)e32, p.lj_inv) * (uint32_t)p.LJ);
     const int64_t r = __ldg(idx + e);
     if (r < 0 || r >= (int64_t)p.P[q]) {
         if (record) record_device_error(kErrIndexRange);

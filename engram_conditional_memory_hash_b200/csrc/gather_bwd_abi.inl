@@ -127,6 +127,9 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     GatherBwdParams p;
     std::memset(&p, 0, sizeof p);
     p.LJ = L * J;
+    // the table of entry e is e mod LJ; its quotient by a reciprocal, exact for
+    // every 32-bit e (the multiplier floor(2^64 / d) + 1, d < 2^32)
+    p.lj_inv = p.LJ == 1 ? 0 : ~uint64_t(0) / (uint64_t)p.LJ + 1;
     p.D = D;
     int64_t R = 0;
     for (int q = 0; q < p.LJ; ++q) {

@@ -192,11 +192,12 @@ def test_empty_and_argument_errors():
         eng.engram_gather_bwd(idx, sizes, d_rows, d_tables, workspace=small)
 
 
-@pytest.mark.parametrize("sizes", [[100, 100], [128, 128], [128, 129], [150, 150, 100], [40000, 30000]])
+@pytest.mark.parametrize("sizes", [[300], [100, 100], [128, 128], [128, 129], [150, 150, 100],
+                                   [40000, 30000]])
 def test_sort_levels(oracle_lib, sizes):
-    # total rows R = 200, 256 (keys of 8 bits: one radix pass), 257 (9 bits:
-    # a second pass on one bit), 400, 70000 (17 bits: three passes); every row
-    # read several times
+    # total rows R = 300 (a single table), 200, 256 (keys of 8 bits: one radix
+    # pass), 257 (9 bits: a second pass on one bit), 400, 70000 (17 bits: three
+    # passes); every row read several times
     r = np.random.default_rng(len(sizes) + sum(sizes))
     sizes = np.array(sizes, dtype=np.int64).reshape(1, -1)
     T, D = 3000, 16
