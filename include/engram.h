@@ -31,7 +31,7 @@
  *     keep their own alignment rules, stated below.
  *   - Errors: arguments are checked before anything is launched; a failing
  *     check returns ENGRAM_ERR_INVALID_ARG (bad pointer, size or alignment) or
- *     ENGRAM_ERR_UNSUPPORTED (a size this build does not handle) and launches
+ *     ENGRAM_ERR_UNSUPPORTED (a size this library does not handle) and launches
  *     nothing.  A failing CUDA runtime call returns ENGRAM_ERR_CUDA.  The
  *     message of the last failure on the calling thread is returned by
  *     engram_last_error().  Kernels never trap; a pipeline wait that exceeds
@@ -301,8 +301,8 @@ ENGRAM_API engram_status_t engram_gate_bwd_fused(const void *grad_out, const voi
  * allocating nothing, for callers that cannot allocate device memory (code
  * that may not call cudaMalloc or an allocating library, e.g. a runtime whose
  * memory policy forbids allocations outside its own pool, or one that only
- * owns the buffers it passes in).  The paper has no counterpart: it is a packaging of the two
- * calls above.
+ * owns the buffers it passes in).  The Engram section has no counterpart: it
+ * is a packaging of the two calls above.
  *
  * Arguments as in engram_gate_bwd, except that the weight-gradient partial
  * rows are kept in a static device array of the library (8 MiB per GPU that
