@@ -10,7 +10,7 @@ constexpr int64_t kGbwdMaxEntries = int64_t(1) << 30;
 // Offsets (bytes, 256-aligned) of the gather backward's scratch in the
 // caller's workspace.  A region zeroed by every call first: the `seen` and
 // `dupmap` bitmaps (one bit per table row) and the counters (list length,
-// listed-chunk count).  Then the unique kernel's per-tile counts, two
+// listed-chunk count).  Then the staging kernel's per-tile counts, two
 // (key, position) buffers for the staged entries, the list and its radix
 // passes (room for every entry), the digit histograms (for the larger of the
 // staged and the list tilings) and totals, and the fp64 partial rows of
@@ -183,12 +183,13 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
         e = launch_pdl(engram::gbwd_mark_kernel, mblocks, (unsigned)engram::kMarkThreads, s, idx, p, seen,
                        dupmap);
     }
+    if (e != cudaSuccess) return cuda_fail(e, "gather_bwd launch");
     // 2. fork: the list kernels (3-5) on the side stream, the unique-row
     //    update on the caller's stream, joined at the end
     std::lock_guard<std::mutex> fork_lock(g_gbwd_mutex);
     GbwdFork *fk = nullptr;
-    if (e == cudaSuccess && (st = gbwd_fork_objects(dev.ordinal, &fk)) != ENGRAM_OK) return st;
-    if (e == cudaSuccess) e = cudaEventRecord(fk->fork, s);
+    if ((st = gbwd_fork_objects(dev.ordinal, &fk)) != ENGRAM_OK) return st;
+    e = cudaEventRecord(fk->fork, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(fk->side, fk->fork, 0);
     if (e != cudaSuccess) return cuda_fail(e, "gather_bwd fork");
     cudaStream_t ls = fk->side;
