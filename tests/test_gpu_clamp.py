@@ -85,3 +85,30 @@ def test_backward_inside_the_clamp(oracle_lib, T, H):
     for name, a, b in zip(("dx", "dk", "dv", "dwh", "dwe"), (dx, dk, dv, dwh, dwe), fused):
         assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), "fused " + name
 
+
+
+@pytest.mark.parametrize("T,H", [(40, 256), (24, 4096), (17, 7168), (19, 1001)])
+def test_zero_fused_weight(oracle_lib, T, H):
+    # wh = 0 makes the fused weight w = wh * we zero, so every token has
+    # dot = 0, s = 0 and gate = 0.5 exactly; then out = x + v/2, and the
+    # backward's dd (inside the clamp, finite) multiplies only terms that are
+    # zero: dx = g and dk = 0 exactly, dv = g/2 exactly, dwe = wh * P = 0;
+    # dwh = we * P is compared with the oracle
+    gi = inputs.gate_inputs(inputs.Workload("zero_w", 500 + H % 11, B=1, S=T, H=H, backward=True))
+    gi["wh"] = np.zeros_like(gi["wh"])
+    t = {n: to_dev_bf16(a) for n, a in gi.items()}
+    out, gate = eng.engram_gate_fwd(t["x"], t["k"], t["v"], t["wh"], t["we"])
+    dx, dk, dv, dwh, dwe = eng.engram_gate_bwd_fused(t["g"], t["x"], t["k"], t["v"], t["wh"], t["we"])
+    torch.cuda.synchronize()
+    assert eng.engram_read_device_error() == 0
+    assert torch.all(gate == 0.5)
+    want_out = (t["x"].float() + 0.5 * t["v"].float()).to(torch.bfloat16)
+    assert torch.equal(out.view(torch.int16), want_out.view(torch.int16))
+    assert torch.equal(dx.view(torch.int16), t["g"].view(torch.int16))
+    assert torch.all(dk.float() == 0.0)
+    assert torch.equal(dv.view(torch.int16), (0.5 * t["g"].float()).to(torch.bfloat16).view(torch.int16))
+    assert torch.all(dwe == 0.0)
+    ref = oracle_lib.engram_gate_bwd(gi["g"], gi["x"], gi["k"], gi["v"], gi["wh"], gi["we"])
+    assert np.all(ref["s"] == 0.0)
+    assert_dw_close("dwh", dwh, ref["dwh"])
+    assert np.abs(ref["dwh"]).max() > 0       # the reduced gradient is not trivially zero
