@@ -242,7 +242,10 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     }
     // 5. segments of the sorted list, then the segments that cross chunks
     const int64_t seg_blocks = (g.nchunks + engram::kSegThreads / 32 - 1) / (engram::kSegThreads / 32);
-    const unsigned blocks = (unsigned)std::min<int64_t>(seg_blocks, int64_t(1) << 30);
+    // at most one wave of segment CTAs (4 per SM), looping over the chunks:
+    // fewer CTAs that find nothing to do compete with the update for SM slots
+    // (155.2 against 156.1 us per call; 2 per SM: 161.3)
+    const unsigned blocks = (unsigned)std::min<int64_t>(seg_blocks, (int64_t)dev.sms * 4);
     const unsigned S_ = engram::kSegThreads;
     const uint32_t *kc = keys[cur], *vc = vals[cur];
     if (e == cudaSuccess) {
@@ -259,8 +262,9 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
             e = launch_pdl(engram::gbwd_segment_kernel<32, 1>, blocks, S_, ls, kc, vc, rows, p, tab4, carry_a,
                            carry_b, carry_list, carry_count, m_c);
     }
-    // one warp per listed chunk (a warp loops when more than 4096 are listed)
-    const int64_t carry_warps = std::min<int64_t>(g.nchunks, 4096);
+    // one warp per listed chunk (a warp loops when more are listed than there
+    // are warps: 8 per SM)
+    const int64_t carry_warps = std::min<int64_t>(g.nchunks, (int64_t)dev.sms * 8);
     const unsigned carry_blocks = (unsigned)((carry_warps + engram::kCarryThreads / 32 - 1) /
                                              (engram::kCarryThreads / 32));
     const unsigned CT = engram::kCarryThreads;
