@@ -284,9 +284,9 @@ __device__ __forceinline__ int64_t list_tiles(uint32_t m)
     return ((int64_t)m + kSortTile - 1) / kSortTile;
 }
 
-// Digit histogram of one tile of the list: hist[digit * ntiles + tile], with
-// ntiles = ceil(M / kSortTile).  Every key of the tile is loaded before any is
-// counted.
+// Digit histograms of the tiles of the list: hist[digit * ntiles + tile], with
+// ntiles = ceil(M / kSortTile); CTA b takes the tiles b, b + gridDim.x, ...
+// Every key of a tile is loaded before any is counted.
 __global__ void __launch_bounds__(kSortThreads)
 gbwd_hist_kernel(const uint32_t *__restrict__ keys, const uint32_t *__restrict__ m_dev, int shift,
                  uint32_t *__restrict__ hist)
@@ -297,20 +297,22 @@ gbwd_hist_kernel(const uint32_t *__restrict__ keys, const uint32_t *__restrict__
     pdl_wait_and_release();
     const uint32_t M = *m_dev;
     const int64_t ntiles = list_tiles(M);
-    if ((int64_t)blockIdx.x >= ntiles) return;
-    const int64_t base = (int64_t)blockIdx.x * kSortTile;
-    uint32_t kk[kSortRounds];
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t base = tile * kSortTile;
+        uint32_t kk[kSortRounds];
 #pragma unroll
-    for (int r = 0; r < kSortRounds; ++r) {
-        const int64_t e = base + r * kSortThreads + tid;
-        kk[r] = e < M ? keys[e] : 0u;
+        for (int r = 0; r < kSortRounds; ++r) {
+            const int64_t e = base + r * kSortThreads + tid;
+            kk[r] = e < M ? keys[e] : 0u;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < kSortRounds; ++r)
+            if (base + r * kSortThreads + tid < M) atomicAdd(&sh[(kk[r] >> shift) & 0xffu], 1u);
+        __syncthreads();
+        hist[(int64_t)tid * ntiles + tile] = sh[tid];
+        sh[tid] = 0;   // the next tile's counts follow the barrier above it
     }
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < kSortRounds; ++r)
-        if (base + r * kSortThreads + tid < M) atomicAdd(&sh[(kk[r] >> shift) & 0xffu], 1u);
-    __syncthreads();
-    hist[(int64_t)tid * ntiles + blockIdx.x] = sh[tid];
 }
 
 // CTA d: exclusive prefix sum of digit d's tile counts hist[d * ntiles ...]
@@ -351,24 +353,25 @@ gbwd_digit_scan_kernel(uint32_t *__restrict__ hist, const uint32_t *__restrict__
     if (tid == 0) totals[blockIdx.x] = carry;
 }
 
-// Stable scatter of one tile of the list by the digit at `shift`.  Round r
-// handles entries base + r * kSortThreads + tid, so (round, warp, lane) is list
-// order.  Within a warp the rank among equal digits comes from
-// __match_any_sync; across the warps of a round, from per-warp digit counts
-// tagged with the round (no clearing between rounds); across rounds, from
-// running digit offsets.  The ranked entries are first placed in shared
+// Stable scatter of the tiles of the list by the digit at `shift`; CTA b
+// takes the tiles b, b + gridDim.x, ...  Round r of a tile handles entries
+// base + r * kSortThreads + tid, so (round, warp, lane) is list order.  Within
+// a warp the rank among equal digits comes from __match_any_sync; across the
+// warps of a round, from per-warp digit counts tagged with the CTA's running
+// round number (no clearing between rounds); across rounds, from running
+// digit offsets.  The ranked entries are first placed in shared
 // memory in digit order, then written out in that order, so that each
 // digit's run of the tile goes to global memory as consecutive words: the
 // run of digit d starts at the digit's base (the sum of all smaller digits'
 // totals) plus this tile's scanned count.  With tile_cnt (the first pass),
-// tile t is the unique kernel's staged tile: tile_cnt[t] entries from
-// t * kSortTile on, one CTA per staged tile.
+// tile t of the staged_tiles tiles is the stage kernel's tile t:
+// tile_cnt[t] entries from t * kSortTile on.
 __global__ void __launch_bounds__(kSortThreads)
 gbwd_scatter_kernel(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
                     const uint32_t *__restrict__ m_dev, const uint32_t *__restrict__ tile_cnt,
                     int shift, const uint32_t *__restrict__ hist,
                     const uint32_t *__restrict__ totals, uint32_t *__restrict__ keys_out,
-                    uint32_t *__restrict__ vals_out)
+                    uint32_t *__restrict__ vals_out, int64_t staged_tiles)
 {
     __shared__ uint32_t gbase[kRadixBins];   // global start of the tile's run of digit d
     __shared__ uint32_t lbase[kRadixBins];   // local start of that run in the tile
@@ -381,92 +384,96 @@ gbwd_scatter_kernel(const uint32_t *__restrict__ keys_in, const uint32_t *__rest
     for (int i = tid; i < kSortWarps * kRadixBins; i += kSortThreads) (&wcnt[0][0])[i] = 0u;
     pdl_wait_and_release();
     const uint32_t M = *m_dev;
-    const int64_t ntiles = tile_cnt != nullptr ? (int64_t)gridDim.x : list_tiles(M);
-    if ((int64_t)blockIdx.x >= ntiles) return;
-    const int64_t base = (int64_t)blockIdx.x * kSortTile;
-    const int n = tile_cnt != nullptr ? (int)min((uint32_t)kSortTile, tile_cnt[blockIdx.x])
-                                      : (int)min((int64_t)kSortTile, (int64_t)M - base);
-    if (n <= 0) return;
+    const int64_t ntiles = tile_cnt != nullptr ? staged_tiles : list_tiles(M);
+    uint32_t iter = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++iter) {
+        __syncthreads();   // nothing of the previous tile is read after this
+        lrun[tid] = 0u;
+        const int64_t base = tile * kSortTile;
+        const int n = tile_cnt != nullptr ? (int)min((uint32_t)kSortTile, tile_cnt[tile])
+                                          : (int)min((int64_t)kSortTile, (int64_t)M - base);
+        if (n <= 0) continue;
 
-    uint32_t kk[kSortRounds], vv[kSortRounds];
+        uint32_t kk[kSortRounds], vv[kSortRounds];
 #pragma unroll
-    for (int r = 0; r < kSortRounds; ++r) {
-        const int e = r * kSortThreads + tid;
-        kk[r] = e < n ? keys_in[base + e] : 0u;
-        vv[r] = e < n ? vals_in[base + e] : 0u;
-    }
-    const uint32_t tot = totals[tid];
-    const uint32_t tile_off = hist[(int64_t)tid * ntiles + blockIdx.x];
-    __syncthreads();
+        for (int r = 0; r < kSortRounds; ++r) {
+            const int e = r * kSortThreads + tid;
+            kk[r] = e < n ? keys_in[base + e] : 0u;
+            vv[r] = e < n ? vals_in[base + e] : 0u;
+        }
+        const uint32_t tot = totals[tid];
+        const uint32_t tile_off = hist[(int64_t)tid * ntiles + tile];
+        __syncthreads();
 #pragma unroll
-    for (int r = 0; r < kSortRounds; ++r)
-        if (r * kSortThreads + tid < n) atomicAdd(&lrun[(kk[r] >> shift) & 0xffu], 1u);
-    __syncthreads();
+        for (int r = 0; r < kSortRounds; ++r)
+            if (r * kSortThreads + tid < n) atomicAdd(&lrun[(kk[r] >> shift) & 0xffu], 1u);
+        __syncthreads();
 
-    // exclusive scans over the digits (thread tid = digit): of the digit
-    // totals for the global base, and of this tile's counts for the local base
-    {
-        const uint32_t cnt = lrun[tid];
-        uint32_t ig = tot, il = cnt;
+        // exclusive scans over the digits (thread tid = digit): of the digit
+        // totals for the global base, and of this tile's counts for the local base
+        {
+            const uint32_t cnt = lrun[tid];
+            uint32_t ig = tot, il = cnt;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t ug = __shfl_up_sync(0xffffffffu, ig, o);
-            const uint32_t ul = __shfl_up_sync(0xffffffffu, il, o);
-            if (lane >= o) {
-                ig += ug;
-                il += ul;
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t ug = __shfl_up_sync(0xffffffffu, ig, o);
+                const uint32_t ul = __shfl_up_sync(0xffffffffu, il, o);
+                if (lane >= o) {
+                    ig += ug;
+                    il += ul;
+                }
             }
-        }
-        if (lane == 31) {
-            warp_sum[0][warp] = ig;
-            warp_sum[1][warp] = il;
-        }
-        __syncthreads();
-        uint32_t bg = 0, bl = 0;
-        for (int w = 0; w < warp; ++w) {
-            bg += warp_sum[0][w];
-            bl += warp_sum[1][w];
-        }
-        gbase[tid] = bg + ig - tot + tile_off;
-        lbase[tid] = bl + il - cnt;
-        lrun[tid] = bl + il - cnt;
-        __syncthreads();
-    }
-
-    const uint32_t below = (1u << lane) - 1u;
-#pragma unroll
-    for (int r = 0; r < kSortRounds; ++r) {
-        const bool valid = r * kSortThreads + tid < n;
-        const uint32_t d = valid ? (kk[r] >> shift) & 0xffu : (uint32_t)kRadixBins;
-        const uint32_t peers = __match_any_sync(0xffffffffu, d);
-        const bool leader = (__ffs(peers) - 1) == lane;
-        const uint32_t tag = (uint32_t)(r + 1) << 8;
-        if (valid && leader) wcnt[warp][d] = tag | (uint32_t)__popc(peers);
-        __syncthreads();
-        if (valid) {
-            uint32_t lp = lrun[d] + (uint32_t)__popc(peers & below);
+            if (lane == 31) {
+                warp_sum[0][warp] = ig;
+                warp_sum[1][warp] = il;
+            }
+            __syncthreads();
+            uint32_t bg = 0, bl = 0;
             for (int w = 0; w < warp; ++w) {
-                const uint32_t c = wcnt[w][d];
-                if ((c & ~0xffu) == tag) lp += c & 0xffu;
+                bg += warp_sum[0][w];
+                bl += warp_sum[1][w];
             }
-            s_key[lp] = kk[r];   // lp < n: the local counts are this tile's own
-            s_val[lp] = vv[r];
+            gbase[tid] = bg + ig - tot + tile_off;
+            lbase[tid] = bl + il - cnt;
+            lrun[tid] = bl + il - cnt;
+            __syncthreads();
+        }
+
+        const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+        for (int r = 0; r < kSortRounds; ++r) {
+            const bool valid = r * kSortThreads + tid < n;
+            const uint32_t d = valid ? (kk[r] >> shift) & 0xffu : (uint32_t)kRadixBins;
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            const bool leader = (__ffs(peers) - 1) == lane;
+            const uint32_t tag = (iter * (uint32_t)kSortRounds + (uint32_t)r + 1u) << 8;
+            if (valid && leader) wcnt[warp][d] = tag | (uint32_t)__popc(peers);
+            __syncthreads();
+            if (valid) {
+                uint32_t lp = lrun[d] + (uint32_t)__popc(peers & below);
+                for (int w = 0; w < warp; ++w) {
+                    const uint32_t c = wcnt[w][d];
+                    if ((c & ~0xffu) == tag) lp += c & 0xffu;
+                }
+                s_key[lp] = kk[r];   // lp < n: the local counts are this tile's own
+                s_val[lp] = vv[r];
+            }
+            __syncthreads();
+            if (valid && leader) atomicAdd(&lrun[d], (uint32_t)__popc(peers));
         }
         __syncthreads();
-        if (valid && leader) atomicAdd(&lrun[d], (uint32_t)__popc(peers));
-    }
-    __syncthreads();
-    for (int i = tid; i < n; i += kSortThreads) {
-        const uint32_t k = s_key[i];
-        const uint32_t d = (k >> shift) & 0xffu;
-        const uint32_t pos = gbase[d] + ((uint32_t)i - lbase[d]);
-        // pos < M whenever the histogram counted the same keys; the check only
-        // keeps every write inside the buffers if that ever failed
-        if (pos < M) {
-            keys_out[pos] = k;
-            vals_out[pos] = s_val[i];
-        } else {
-            record_device_error(kErrIndexRange);
+        for (int i = tid; i < n; i += kSortThreads) {
+            const uint32_t k = s_key[i];
+            const uint32_t d = (k >> shift) & 0xffu;
+            const uint32_t pos = gbase[d] + ((uint32_t)i - lbase[d]);
+            // pos < M whenever the histogram counted the same keys; the check only
+            // keeps every write inside the buffers if that ever failed
+            if (pos < M) {
+                keys_out[pos] = k;
+                vals_out[pos] = s_val[i];
+            } else {
+                record_device_error(kErrIndexRange);
+            }
         }
     }
 }
