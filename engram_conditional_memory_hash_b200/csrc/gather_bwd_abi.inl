@@ -179,7 +179,7 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     // 1. mark rows read more than once
     if (e == cudaSuccess) {
         const unsigned mblocks = (unsigned)std::min<int64_t>(
-            (N + 4 * engram::kMarkThreads - 1) / (4 * engram::kMarkThreads), 4096);
+            (N + engram::kMarkThreads - 1) / engram::kMarkThreads, 16384);
         e = launch_pdl(engram::gbwd_mark_kernel, mblocks, (unsigned)engram::kMarkThreads, s, idx, p, seen,
                        dupmap);
     }
