@@ -194,15 +194,14 @@ engram_status_t engram_gather_bwd(const int64_t *idx, int64_t T, int32_t L, int3
     if (e != cudaSuccess) return cuda_fail(e, "gather_bwd fork");
     cudaStream_t ls = fk->side;
     // the rows read once: updated in place on the caller's stream, one CTA per
-    // tile of entries (short-lived CTAs, so that the list kernels find slots)
+    // tile of entries (short-lived CTAs, so that the list kernels find slots);
+    // a programmatic dependent of the mark kernel, so that its first CTAs are
+    // resident when the mark completes (145.8 against 147.4 us per call)
     {
         const unsigned ub = (unsigned)((N + engram::kUpdTile - 1) / engram::kUpdTile);
         const unsigned ut = (unsigned)engram::kUpdThreads;
         const uint32_t *dm = dupmap;
-        auto uniq = [&](auto kern) {
-            kern<<<ub, ut, 0, s>>>(idx, rows, p, dm, tab4);
-            return cudaGetLastError();
-        };
+        auto uniq = [&](auto kern) { return launch_pdl(kern, ub, ut, s, idx, rows, p, dm, tab4); };
         e = nv <= 4 ? uniq(engram::gbwd_unique_kernel<4, 2>)
           : nv <= 8 ? uniq(engram::gbwd_unique_kernel<8, 2>)
           : nv <= 16 ? uniq(engram::gbwd_unique_kernel<16, 2>)
