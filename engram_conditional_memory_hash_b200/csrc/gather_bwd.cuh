@@ -43,9 +43,10 @@
 // gradients enter the fp64 sums exactly; the row's fp32 value is updated with
 // one rounding: d_tables[r] = fp32((double)d_tables[r] + sum).
 //
-// The length M of the list exists only on the device, so the list kernels are
-// launched for the worst case (M = N) and read M first: CTAs and warps beyond
-// it return at once.
+// The length M of the list exists only on the device, so the list kernels'
+// grids are fixed on the host (sized for the worst case, M = N, or capped and
+// looping over the work) and read M first: CTAs and warps beyond it return at
+// once.
 #pragma once
 
 #include "common.cuh"
