@@ -417,3 +417,41 @@ def test_side_stream_in_cuda_graph():
     assert eng.engram_read_device_error() == 0
     assert _bits_equal(t, want)
     del g
+
+
+@pytest.mark.parametrize("repeated", [1024, 1025, 2048, 4097, 64 * 37])
+def test_list_lengths_at_tile_edges(oracle_lib, repeated):
+    # exactly `repeated` entries fall on rows read more than once (pairs, plus
+    # one triple when the count is odd), the other entries on rows read once:
+    # the sorted list then fills whole radix tiles of 1024 entries, or spills
+    # one entry into the next tile, or whole segment chunks of 64 entries
+    r = np.random.default_rng(repeated)
+    L, J, D = 1, 4, 16
+    sizes = np.full((L, J), 200003, dtype=np.int64)
+    T = 6000
+    n = T * L * J
+    tab = np.tile(np.arange(J), T)                 # entry e belongs to table e % J
+    rows = np.empty(n, dtype=np.int64)
+    # distinct rows per table for every entry first
+    for j in range(J):
+        sel = np.flatnonzero(tab == j)
+        rows[sel] = r.choice(200003, size=sel.size, replace=False)
+    # then make `repeated` entries share rows: pairs of entries of the same
+    # table read the same row (a triple if the count is odd)
+    pick = r.choice(np.flatnonzero(tab == 0), size=repeated, replace=False)
+    k = 0
+    while k < repeated:
+        take = 3 if repeated - k == 3 else 2
+        rows[pick[k:k + take]] = rows[pick[k]]
+        k += take
+    idx_np = rows.reshape(T, L, J)
+    first = np.concatenate([[0], np.cumsum(sizes.ravel())[:-1]])
+    keys = (idx_np.reshape(-1, L * J) + first[None]).ravel()
+    _, inv, cnt = np.unique(keys, return_inverse=True, return_counts=True)
+    assert int((cnt[inv] > 1).sum()) == repeated
+    d_rows = inputs.f32_to_bf16_bits(r.standard_normal((T, L, J, D)).astype(np.float32))
+    R = int(sizes.sum())
+    init = np.zeros((R, D))
+    got = _run(torch.from_numpy(idx_np).cuda(), sizes, d_rows, init)
+    want, tol, touched = _expect(oracle_lib, idx_np, sizes, d_rows, init)
+    _check(got, want, tol, touched, init)
