@@ -430,7 +430,7 @@ def run_ours(args):
         uniq = int(torch.unique(buf0.idx.view(T, L * J) + first[None]).numel())
         us = time_calls(lambda: eng.engram_gather_bwd(buf0.idx, hin["table_sizes"], d_rows,
                                                       d_tables, workspace=ws, stream=stream),
-                        stream, dev, warmup=3, calls=20)
+                        stream, dev, warmup=5, calls=100)
         # idx read + d_rows read + one read and one write of every touched fp32 table row
         gbwd = kernel_entry(us, gather_bwd_bytes(T, L, J, D, uniq), peak)
         gbwd.update({"traffic": committed_traffic("gather_bwd", T), "unique_rows": uniq,
@@ -438,7 +438,7 @@ def run_ours(args):
                      "what": "engram_gather_bwd on the step's indices: rows read once updated "
                              "in place, the rest listed, radix-sorted by row and summed in fp64 "
                              "on a side stream beside the update; fp32 table-gradient update; "
-                             "20 calls back to back, CUDA events around them"})
+                             "100 calls back to back after 5, CUDA events around them"})
         del d_rows, d_tables, ws
 
     kern = {n: kernel_entry(per_kernel_ms[n] * 1e3, ab[n], peak) for n in names}
