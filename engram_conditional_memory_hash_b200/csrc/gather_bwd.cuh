@@ -73,7 +73,7 @@ constexpr int kUpdThreads = 64;                         // unique-row update
 constexpr int kUpdWarpEntries = 32;                     // entries per warp in the update
 constexpr int kUpdTile = kUpdThreads / 32 * kUpdWarpEntries;
 static_assert(kSortThreads == kRadixBins, "one thread per digit in the histogram epilogue");
-static_assert(kUniqTile == kSortTile, "the first radix pass reads the unique kernel's staged tiles");
+static_assert(kUniqTile == kSortTile, "the first radix pass reads the stage kernel's tiles");
 
 struct GatherBwdParams {
     int64_t N;                          // entries: T * L * J
@@ -313,7 +313,7 @@ gbwd_hist_kernel(const uint32_t *__restrict__ keys, const uint32_t *__restrict__
 
 // CTA d: exclusive prefix sum of digit d's tile counts hist[d * ntiles ...]
 // in place, and the digit's total in totals[d].  ntiles = staged_tiles for
-// the first pass (the unique kernel's tiles), else ceil(M / kSortTile).
+// the first pass (the stage kernel's tiles), else ceil(M / kSortTile).
 __global__ void __launch_bounds__(kScanThreads)
 gbwd_digit_scan_kernel(uint32_t *__restrict__ hist, const uint32_t *__restrict__ m_dev,
                        int64_t staged_tiles, uint32_t *__restrict__ totals)
